@@ -1,0 +1,85 @@
+"""Plant mistakes in copies of the oracle's C file and check that the pins
+catch every one: evidence that the pins constrain each step of the oracle
+(rounding, scale, zero point, range widening, clamp, packing map, decoding,
+linear indexing).  Everything runs on the CPU."""
+from __future__ import annotations
+
+import os
+import subprocess
+
+import numpy as np
+import pytest
+
+from oracle import oracle as O
+import tests.test_oracle_pins as P
+
+MUTANTS = {
+    "round_half_away": ("int r = (int)nearbyintf(t);", "int r = (int)roundf(t);"),
+    "zero_round_half_away": ("int z = (int)nearbyintf(zq);", "int z = (int)roundf(zq);"),
+    "levels_2^b": ("float s = range / (float)qmax;", "float s = range / (float)(qmax + 1);"),
+    "no_zero_in_range": ("if (lo > 0.0f) lo = 0.0f;", ""),
+    "zero_sign": ("float zq = -lo / s;", "float zq = lo / s;"),
+    "reciprocal_multiply": ("float t = x[i] / s;", "float t = x[i] * (1.0f / s);"),
+    "no_clamp": ("if (q > qmax) q = qmax;", ""),
+    "lane_transposed": ("int lane = 4 * r + c;", "int lane = 4 * c + r;"),
+    "nibble_pairing": ("field = slot + 4 * odd;", "field = 2 * slot + odd;"),
+    "crumb_run_offset": ("field = 4 * (run % 2) + slot + 8 * odd;", "field = 8 * (run % 2) + slot + 4 * odd;"),
+    "linear_zero_sign": ("wrow[k] = (double)((int)codes[n * K + k] - (int)zeros[n * G + j])",
+                         "wrow[k] = (double)((int)codes[n * K + k] + (int)zeros[n * G + j])"),
+    "linear_scale_transposed": ("* (double)scales[n * G + j];\n        }\n        for (int64_t m",
+                                "* (double)scales[j * N + n];\n        }\n        for (int64_t m"),
+    "f16_bias": ("mag = ldexpf((float)(1024 + f), e - 25);", "mag = ldexpf((float)(1024 + f), e - 24);"),
+    "f16_subnormal": ("mag = ldexpf((float)f, -24);", "mag = ldexpf((float)f, -25);"),
+}
+
+# cheap pins first; each mutant only has to fail one of them
+PINS = [
+    (P.test_worked_examples, {"name": "int4_g8_worked.txt"}),
+    (P.test_worked_examples, {"name": "int2_g8_worked.txt"}),
+    (P.test_worked_examples, {"name": "int4_clamp_worked.txt"}),
+    (P.test_worked_examples, {"name": "int4_zero_tie_worked.txt"}),
+    (P.test_page_scale_example, {}),
+    (P.test_constant_groups, {}),
+    (P.test_interleaved_positions_hand_derived, {}),
+    (P.test_decode_f16_all_patterns, {}),
+    (P.test_invariants, {"bits": 4, "g": 32}),
+    (P.test_linear_closed_form, {"bits": 4, "g": 128}),
+    (P.test_brute_force_optimal_codes, {"bits": 2}),
+    (P.test_exact_rational_arithmetic, {}),
+]
+
+
+def _build_mutant(tmp_path, name):
+    src = open(os.path.join(os.path.dirname(O.__file__), "bq_oracle.c")).read()
+    old, new = MUTANTS[name]
+    assert src.count(old) == 1, f"mutation site for {name} not unique/found"
+    c = tmp_path / f"{name}.c"
+    c.write_text(src.replace(old, new))
+    so = tmp_path / f"{name}.so"
+    subprocess.check_call(["gcc", *O.CFLAGS, str(c), "-o", str(so), "-lm"])
+    return str(so)
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(tmp_path, name):
+    so = _build_mutant(tmp_path, name)
+    caught = None
+    with O.using_library(so):
+        for fn, kw in PINS:
+            try:
+                fn(**kw)
+            except (AssertionError, O.OracleError):
+                caught = fn.__name__
+                break
+    assert caught is not None, f"mutant {name} passed every pin"
+
+
+def test_unmutated_copy_passes(tmp_path):
+    src = open(os.path.join(os.path.dirname(O.__file__), "bq_oracle.c")).read()
+    c = tmp_path / "same.c"
+    c.write_text(src)
+    so = tmp_path / "same.so"
+    subprocess.check_call(["gcc", *O.CFLAGS, str(c), "-o", str(so), "-lm"])
+    with O.using_library(str(so)):
+        for fn, kw in PINS:
+            fn(**kw)

@@ -1,0 +1,400 @@
+"""Pins for the CPU oracle: checks against values and properties that the pages
+and the mathematics fix, none of which re-types the oracle's own formulas.
+
+  * hand-worked examples with dyadic values (tests/golden/*.txt)
+  * the page's 8-bit scale example ("大模型量化实战" section 2.2)
+  * invariants: code range, |x - dequant| <= s/2, group ends within s/2
+  * constant groups, one-signed groups, the all-zero group
+  * optimality brute force: each code is a nearest grid point, ties to even
+  * exact rational arithmetic for the fp32 steps (independent rounding code)
+  * packing: hand-derived positions, bijection, canonical word examples
+  * element decoding against numpy / torch conversions
+  * the linear layer against a closed form and an exactly-rounded sum
+"""
+from __future__ import annotations
+
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def read_golden(name):
+    d = {}
+    with open(os.path.join(GOLD, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, *vals = line.split()
+            d[key] = vals
+    return d
+
+
+# --------------------------------------------------------------------------
+# independent exact arithmetic (Fractions) for IEEE binary32 round-to-nearest
+# --------------------------------------------------------------------------
+
+def rne_int(q: Fraction) -> int:
+    n = math.floor(q)
+    rem = q - n
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and n % 2 == 1):
+        n += 1
+    return n
+
+
+def rne_f32(q: Fraction) -> Fraction:
+    """Round a rational to the nearest binary32 value (ties to even), exactly."""
+    if q == 0:
+        return Fraction(0)
+    sign = -1 if q < 0 else 1
+    a = abs(q)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    qe = max(e - 23, -149)
+    n = rne_int(a / Fraction(2) ** qe)
+    return sign * Fraction(n) * Fraction(2) ** qe
+
+
+def exact_group(x32: np.ndarray, bits: int):
+    """The quantizer's steps (reading R1-R3) in exact rational arithmetic."""
+    qmax = (1 << bits) - 1
+    xs = [Fraction(float(v)) for v in x32]
+    lo = min(min(xs), Fraction(0))
+    hi = max(max(xs), Fraction(0))
+    s = rne_f32(rne_f32(hi - lo) / qmax)
+    if s == 0:
+        return 0.0, 0, [0] * len(xs)
+    z = rne_int(rne_f32(-lo / s))
+    q = [min(max(rne_int(rne_f32(v / s)) + z, 0), qmax) for v in xs]
+    return float(s), z, q
+
+
+# --------------------------------------------------------------------------
+# worked examples
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", ["int4_g8_worked.txt", "int2_g8_worked.txt", "int4_clamp_worked.txt",
+                                  "int4_zero_tie_worked.txt"])
+def test_worked_examples(name):
+    g = read_golden(name)
+    bits = int(g["bits"][0])
+    x = np.array([float(v) for v in g["x"]], dtype=np.float32)
+    s, z, q = O.quantize_group(x, bits)
+    assert s == float(g["s"][0])
+    assert z == int(g["z"][0])
+    assert q.tolist() == [int(v) for v in g["q"]]
+    deq = (q.astype(np.float64) - z) * s
+    assert deq.tolist() == [float(v) for v in g["dequant"]]
+    for key in ("canonical_word32", "canonical_word16"):
+        if key in g:
+            packed = O.pack(q.reshape(1, -1), bits, "canonical")
+            assert int.from_bytes(packed.tobytes(), "little") == int(g[key][0], 16)
+
+
+def test_page_scale_example():
+    g = read_golden("page_scale_example.txt")
+    x = np.array([float(v) for v in g["x"]], dtype=np.float32)
+    s, z, q = O.quantize_group(x, int(g["bits"][0]))
+    assert abs(s - float(g["s_approx"][0])) < float(g["s_abs_tol"][0])
+    assert z == int(g["z"][0])
+    assert q.tolist() == [int(v) for v in g["q"]]
+
+
+# --------------------------------------------------------------------------
+# invariants and special groups
+# --------------------------------------------------------------------------
+
+def _random_groups(rng, count, g):
+    kinds = []
+    for i in range(count):
+        k = i % 7
+        if k == 0:
+            v = rng.normal(0, 0.02, g)
+        elif k == 1:
+            v = rng.standard_t(4, g) * 0.01
+        elif k == 2:
+            v = np.abs(rng.normal(0, 1, g)) + 0.1          # one-signed positive
+        elif k == 3:
+            v = -np.abs(rng.normal(0, 1, g)) - 0.1         # one-signed negative
+        elif k == 4:
+            v = rng.integers(-8, 9, g) * 0.125             # dyadic grid: many ties
+        elif k == 5:
+            v = rng.normal(0, 1, g)
+            v[rng.integers(0, g)] *= 50.0                  # one outlier
+        else:
+            v = rng.uniform(-3, 7, g)
+        kinds.append(v.astype(np.float16).astype(np.float32))
+    return kinds
+
+
+@pytest.mark.parametrize("bits,g", [(4, 128), (2, 64), (4, 32), (2, 8)])
+def test_invariants(bits, g):
+    rng = np.random.default_rng(1000 + bits * 7 + g)
+    qmax = (1 << bits) - 1
+    for x in _random_groups(rng, 300, g):
+        s, z, q = O.quantize_group(x, bits)
+        assert 0 <= z <= qmax
+        assert q.min() >= 0 and q.max() <= qmax
+        deq = (q.astype(np.float64) - z) * s
+        err = np.abs(deq - x.astype(np.float64))
+        bound = s / 2 + s * 2.0 ** -18
+        assert err.max() <= bound, (err.max(), s)
+        # the two ends of the (zero-widened) range reconstruct within s/2
+        i_lo, i_hi = int(np.argmin(x)), int(np.argmax(x))
+        assert err[i_lo] <= bound and err[i_hi] <= bound
+
+
+def test_constant_groups():
+    # all zero: the guarded case, s = 0
+    s, z, q = O.quantize_group(np.zeros(64, np.float32), 2)
+    assert (s, z) == (0.0, 0) and not q.any()
+    s, z, q = O.quantize_group(-np.zeros(16, np.float32), 4)
+    assert (s, z) == (0.0, 0) and not q.any()
+    # constant c != 0 reconstructs c within fp32 rounding
+    for c in (0.75, -0.75, 3.0e-3, -1.0e4):
+        for bits in (2, 4):
+            qmax = (1 << bits) - 1
+            s, z, q = O.quantize_group(np.full(32, c, np.float32), bits)
+            assert s > 0
+            deq = (int(q[0]) - z) * s
+            assert abs(deq - c) <= abs(c) * 2.0 ** -20
+            assert len(set(q.tolist())) == 1
+            if c > 0:
+                assert z == 0 and q[0] == qmax
+            else:
+                assert z == qmax and q[0] == 0
+
+
+def test_nonfinite_rejected():
+    for bad in (np.inf, -np.inf, np.nan):
+        x = np.zeros(8, np.float32)
+        x[3] = bad
+        with pytest.raises(O.OracleError):
+            O.quantize_group(x, 4)
+
+
+# --------------------------------------------------------------------------
+# brute force
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_brute_force_optimal_codes(bits):
+    """Every code is a nearest point of the grid {(q - z) s}, ties to an even
+    (q - z), except where the quotient sits within fp32 rounding of a tie."""
+    qmax = (1 << bits) - 1
+    vals = [Fraction(k, 8) for k in range(-12, 13)]
+    rng = np.random.default_rng(7 + bits)
+    for g in (2, 3, 4):
+        for _ in range(400):
+            xs = [vals[i] for i in rng.integers(0, len(vals), g)]
+            x32 = np.array([float(v) for v in xs], np.float32)
+            s, z, q = O.quantize_group(x32, bits)
+            if s == 0:
+                assert all(v == 0 for v in xs) and not q.any()
+                continue
+            S = Fraction(s)
+            for xi, qi in zip(xs, q.tolist()):
+                d = [abs((c - z) * S - xi) for c in range(qmax + 1)]
+                best = min(d)
+                cand = [c for c in range(qmax + 1) if d[c] == best]
+                t = xi / S
+                near_tie = abs((t - math.floor(t)) - Fraction(1, 2)) < Fraction(1, 2 ** 18)
+                if near_tie and len(cand) == 1:
+                    assert abs(qi - cand[0]) <= 1
+                    continue
+                assert qi in cand, (xs, s, z, q)
+                if len(cand) == 2:
+                    assert (qi - z) % 2 == 0
+
+
+def test_exact_rational_arithmetic():
+    """The fp32 steps agree with exact rational arithmetic followed by
+    round-to-nearest-even, including constructed near-tie quotients."""
+    rng = np.random.default_rng(99)
+    groups = _random_groups(rng, 140, 16)
+    # near ties: x = fp32 nearest to (k + 1/2) s, plus its neighbours
+    for _ in range(200):
+        bits = 4
+        base = rng.normal(0, 1, 16).astype(np.float32)
+        s_guess = np.float32((base.max() - min(base.min(), 0)) / 15)
+        k = int(rng.integers(-7, 8))
+        t = np.float32((k + 0.5) * float(s_guess))
+        nb = np.nextafter(t, np.float32(np.inf)), np.nextafter(t, np.float32(-np.inf))
+        base[3], base[5], base[7] = t, nb[0], nb[1]
+        groups.append(base.astype(np.float32))
+    for i, x in enumerate(groups):
+        for bits in (2, 4):
+            s, z, q = O.quantize_group(x, bits)
+            es, ez, eq = exact_group(x, bits)
+            assert (s, z, q.tolist()) == (es, ez, eq), (i, bits)
+
+
+# --------------------------------------------------------------------------
+# matrix-level quantize (row/group indexing, fp16 and bf16 inputs)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("wtype", ["f16", "bf16"])
+def test_matrix_quantize_matches_groups(wtype):
+    rng = np.random.default_rng(5)
+    N, K, g = 6, 256, 64
+    w = torch.from_numpy(rng.normal(0, 0.02, (N, K)).astype(np.float32)).to(
+        torch.float16 if wtype == "f16" else torch.bfloat16)
+    bits16 = w.view(torch.int16).numpy().view(np.uint16)
+    codes, scales, zeros = O.quantize(bits16, wtype, 2, g, threads=3)
+    wf = w.float().numpy()
+    for n in range(N):
+        for j in range(K // g):
+            s, z, q = O.quantize_group(wf[n, j * g:(j + 1) * g], 2)
+            assert scales[n, j] == np.float32(s) and zeros[n, j] == z
+            assert (codes[n, j * g:(j + 1) * g] == q).all()
+
+
+# --------------------------------------------------------------------------
+# element decoding and bf16 rounding
+# --------------------------------------------------------------------------
+
+def test_decode_f16_all_patterns():
+    pats = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    mine = O.decode_f64(pats, "f16")
+    ref = pats.view(np.float16).astype(np.float64)
+    both_nan = np.isnan(mine) & np.isnan(ref)
+    assert ((mine == ref) | both_nan).all()
+    assert (np.signbit(mine) == np.signbit(ref))[~both_nan].all()
+
+
+def test_decode_bf16_all_patterns():
+    pats = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    mine = O.decode_f64(pats, "bf16")
+    ref = torch.from_numpy(pats.view(np.int16)).view(torch.bfloat16).double().numpy()
+    both_nan = np.isnan(mine) & np.isnan(ref)
+    assert ((mine == ref) | both_nan).all()
+
+
+def test_bf16_rounding():
+    rng = np.random.default_rng(3)
+    v = rng.normal(0, 10, 4000).astype(np.float32).astype(np.float64)
+    mine = O.to_bf16_bits(v)
+    ref = torch.from_numpy(v.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert (mine == ref).all()
+    # direct rounding of doubles: an exact tie goes to even, just above goes up
+    assert O.to_bf16_bits(np.array([1 + 2 ** -8]))[0] == 0x3F80
+    assert O.to_bf16_bits(np.array([1 + 2 ** -8 + 2 ** -40]))[0] == 0x3F81
+    assert O.to_bf16_bits(np.array([1 + 3 * 2 ** -8]))[0] == 0x3F82
+    assert O.to_bf16_bits(np.array([-2.0]))[0] == 0xC000
+
+
+# --------------------------------------------------------------------------
+# packing
+# --------------------------------------------------------------------------
+
+def test_interleaved_positions_hand_derived():
+    with open(os.path.join(GOLD, "interleaved_positions.txt")) as f:
+        rows = [l.split() for l in f if l.strip() and not l.startswith("#")]
+    assert len(rows) >= 16
+    for bits, cols, n, k, byte, bit in (map(int, r) for r in rows):
+        assert O.code_position("interleaved", n, k, cols, bits) == (byte, bit), (bits, cols, n, k)
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+@pytest.mark.parametrize("layout", ["canonical", "interleaved"])
+def test_pack_bijection(bits, layout):
+    N, K = 32, 256
+    rng = np.random.default_rng(bits)
+    seen = set()
+    for n in range(N):
+        for k in range(K):
+            seen.add(O.code_position(layout, n, k, K, bits))
+    assert len(seen) == N * K
+    assert all(0 <= b < N * K * bits // 8 and o % bits == 0 and o < 8 for b, o in seen)
+    codes = rng.integers(0, 1 << bits, (N, K), dtype=np.uint8)
+    p = O.pack(codes, bits, layout)
+    assert p.size == N * K * bits // 8
+    assert (O.unpack(p, N, K, bits, layout) == codes).all()
+
+
+def test_canonical_is_row_major_lsb_first():
+    codes = np.array([[1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11, 12, 13, 14, 15, 0]], np.uint8)
+    p = O.pack(codes, 4, "canonical")
+    assert p.tobytes() == bytes([0x21, 0x43, 0x65, 0x87, 0xA9, 0xCB, 0xED, 0x0F])
+    c2 = np.array([[3, 0, 1, 2] * 4], np.uint8)
+    assert O.pack(c2, 2, "canonical").tobytes() == bytes([0b10010011] * 4)
+
+
+def test_storage_sizes_match_page():
+    # "低比特量化": a 70B-parameter model takes 35 GB at INT4 and 17.5 GB at INT2
+    # (codes only, 1 GB = 1e9 bytes)
+    for bits, gb in ((4, 35.0), (2, 17.5)):
+        assert 70e9 * bits / 8 / 1e9 == gb
+
+
+# --------------------------------------------------------------------------
+# linear
+# --------------------------------------------------------------------------
+
+def _representable_matrix(rng, N, K, g, bits):
+    """W whose groups are reproduced exactly by the quantizer: per group a
+    power-of-two scale, a zero point, and codes that include both 0 and
+    2^b - 1 so the range is exactly (2^b - 1) s."""
+    qmax = (1 << bits) - 1
+    G = K // g
+    codes = rng.integers(0, qmax + 1, (N, K)).astype(np.uint8)
+    for n in range(N):
+        for j in range(G):
+            i0, i1 = rng.choice(g, 2, replace=False)
+            codes[n, j * g + i0] = 0
+            codes[n, j * g + i1] = qmax
+    zeros = rng.integers(0, qmax + 1, (N, G)).astype(np.uint8)
+    scales = np.float32(2.0) ** rng.integers(-9, -4, (N, G)).astype(np.float32)
+    W = np.empty((N, K), np.float64)
+    for n in range(N):
+        for j in range(G):
+            W[n, j * g:(j + 1) * g] = (codes[n, j * g:(j + 1) * g].astype(np.float64) - zeros[n, j]) * scales[n, j]
+    return W, codes, scales, zeros
+
+
+@pytest.mark.parametrize("bits,g", [(4, 128), (2, 64)])
+def test_linear_closed_form(bits, g):
+    rng = np.random.default_rng(11 * bits)
+    N, K, M = 24, 512, 5
+    W, codes, scales, zeros = _representable_matrix(rng, N, K, g, bits)
+    w16 = W.astype(np.float16)
+    assert (w16.astype(np.float64) == W).all()
+    c2, s2, z2 = O.quantize(w16.view(np.uint16), "f16", bits, g)
+    assert (c2 == codes).all() and (s2 == scales).all() and (z2 == zeros).all()
+    assert (O.dequant_f64(c2, s2, z2, g) == W).all()
+    x = rng.normal(0, 1, (M, K)).astype(np.float16).astype(np.float64)
+    y = O.linear_f64(x, c2, s2, z2, g, threads=2)
+    ref = x @ W.T
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_linear_exact_sum():
+    rng = np.random.default_rng(2)
+    N, K, M, g = 4, 64, 3, 32
+    w = rng.normal(0, 0.02, (N, K)).astype(np.float16)
+    codes, scales, zeros = O.quantize(w.view(np.uint16), "f16", 4, g)
+    x = rng.normal(0, 1, (M, K)).astype(np.float16).astype(np.float64)
+    y = O.linear_f64(x, codes, scales, zeros, g)
+    for m in range(M):
+        for n in range(N):
+            terms = [x[m, k] * ((int(codes[n, k]) - int(zeros[n, k // g])) * float(scales[n, k // g]))
+                     for k in range(K)]
+            exact = math.fsum(terms)
+            assert abs(y[m, n] - exact) <= 1e-13 * math.fsum(abs(t) for t in terms) + 1e-300
+
+
+def test_mixed_offsets_hand_computed():
+    code_off, group_off = O.mixed_offsets([4, 2, 4], 256)
+    assert code_off == [0, 16384, 24576, 40960]
+    assert group_off == [0, 256, 768, 1024]
