@@ -1,0 +1,532 @@
+#!/usr/bin/env python
+"""Benchmark of the W4/W2 weight-only decode path on a Llama-3-8B-shaped stack.
+
+One step = one decode forward through all 32 layers x 7 linears
+(q, k, v, o 4096x4096 / 1024x4096; gate, up 14336x4096; down 4096x14336)
+for each batch size M in {1, 4, 16}: 672 bq_linear calls, replayed from one
+CUDA graph.  Weights are synthetic fp16 N(0, 0.02) (seed 1000*layer + module),
+quantized on the GPU by bq_quantize (INT4 group 128 by default); activations
+are bf16 N(0, 1).  The packed stack (3.76 GB at INT4) is far larger than the
+126 MB L2, so every pass streams the weights from HBM; no flush is needed.
+
+Printed: ONE JSON line (rank 0).  ``value`` = effective weight GB/s of the
+whole job = (packed codes + scales + zeros + x + y bytes of every linear of
+the step, over all ranks) / max-over-ranks step time.  Extra fields report
+per-M numbers, per-shape numbers, the quantizer over the whole ~7B-weight
+stack, the end-to-end host-buffer path, the roofline of the dominant kernel
+(the decode GEMV) and the CPU oracle baseline.
+
+Multi-GPU (torchrun): every rank runs its own replica of the stack on its own
+GPU with its own inputs (independent batches, no data-path collective);
+``scaling`` is "weak".
+
+``--impl reference`` times the CPU oracle (the plain C reference of the same
+computation) on a bounded sample of the same workload, on this host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from quantized_gemm_group_b200 import bq, synth  # noqa: E402
+
+MEASURED_PEAKS = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+M_SET = (1, 4, 16)
+METRIC = "W4/W2 dequant-GEMV weight GB/s (M<=16) & GEMM TFLOP/s (M>=2048) vs roofline"
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+
+def weight_bytes(N, K, bits, group):
+    """Algorithmic bytes of one decode linear's weights: codes + fp32 scale + u8 zero."""
+    return N * K * bits // 8 + N * (K // group) * 5
+
+
+def linear_bytes(N, K, bits, group, M):
+    return weight_bytes(N, K, bits, group) + 2 * M * K + 2 * M * N
+
+
+def peaks():
+    try:
+        with open(MEASURED_PEAKS) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", 0)), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        out = {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        if not self.path or not os.path.exists(self.path):
+            return out
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        if sm:
+            busy = [s for s in sm if s > 0.5 * max(sm)] or sm
+            out = {"sm_mhz": statistics.median(busy), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                   "samples": len(sm)}
+        return out
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() and dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def stack_shapes(layers):
+    return [(l, mi, name, N, K) for l in range(layers) for mi, (name, N, K) in enumerate(synth.LLAMA3_8B_LINEARS)]
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+class Stack:
+    """The quantized decode stack resident in HBM, plus per-M activations."""
+
+    def __init__(self, layers, bits, group, seed_offset, dist_kind, quant_time=True):
+        self.layers, self.bits, self.group = layers, bits, group
+        self.shapes = stack_shapes(layers)
+        dev = "cuda"
+        # fp16 weights for the whole stack (~14 GB at 32 layers) so the
+        # quantizer can be timed over all of it, then dropped.
+        Ws = []
+        for (l, mi, name, N, K) in self.shapes:
+            seed = synth.weight_seed(l, mi) + seed_offset
+            if dist_kind == "t4":
+                Ws.append(synth.student_t4((N, K), 0.02, seed, "f16", dev, outlier_frac=0.001))
+            else:
+                Ws.append(synth.normal((N, K), 0.02, seed, "f16", dev))
+        self.q = []
+        for W, (l, mi, name, N, K) in zip(Ws, self.shapes):
+            self.q.append(bq.bq_quantize(W, bits, group, "interleaved"))
+        torch.cuda.synchronize()
+        if bq.bq_device_status() != bq.BQ_OK:
+            raise RuntimeError("quantizer reported a device error")
+        self.quant = None
+        if quant_time:
+            self.quant = self._time_quantizer(Ws)
+        del Ws
+        torch.cuda.empty_cache()
+
+    def _time_quantizer(self, Ws, reps=3):
+        """Quantize the whole stack (all ~7B weights) from one CUDA graph."""
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            for W, out in zip(Ws, self.q):            # warm
+                bq.bq_quantize(W, self.bits, self.group, "interleaved", out=out, stream=s)
+            s.synchronize()
+            with torch.cuda.graph(g, stream=s):
+                for W, out in zip(Ws, self.q):
+                    bq.bq_quantize(W, self.bits, self.group, "interleaved", out=out, stream=s)
+        torch.cuda.current_stream().wait_stream(s)
+        g.replay()
+        torch.cuda.synchronize()
+        times = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            g.replay()
+            b.record()
+            b.synchronize()
+            times.append(a.elapsed_time(b) / 1e3)
+        t = min(times)
+        weights = sum(N * K for (_, _, _, N, K) in self.shapes)
+        byts = sum(N * K * 2 + weight_bytes(N, K, self.bits, self.group) for (_, _, _, N, K) in self.shapes)
+        del g
+        return {"weights": weights, "seconds": t, "weights_per_s": weights / t, "GBps": byts / t / 1e9,
+                "bytes": byts, "launches": len(self.shapes)}
+
+    def make_graph(self, Ms, xs, ys, stream):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            for M in Ms:                                  # warm / lazy init outside capture
+                for i, (l, mi, name, N, K) in enumerate(self.shapes):
+                    pk, sc, ze = self.q[i]
+                    bq.bq_linear(xs[M][i], pk, sc, ze, N, self.bits, self.group, out=ys[M][i], stream=stream)
+            stream.synchronize()
+            with torch.cuda.graph(g, stream=stream):
+                for M in Ms:
+                    for i, (l, mi, name, N, K) in enumerate(self.shapes):
+                        pk, sc, ze = self.q[i]
+                        bq.bq_linear(xs[M][i], pk, sc, ze, N, self.bits, self.group, out=ys[M][i], stream=stream)
+        return g
+
+    def step_bytes(self, Ms):
+        return sum(linear_bytes(N, K, self.bits, self.group, M) for M in Ms for (_, _, _, N, K) in self.shapes)
+
+
+def time_graph(g, steps, warmup, stream, world, profile=False):
+    """Replay `g` warmup + steps times; the steps are timed with CUDA events on
+    `stream`.  profile=True brackets the timed replays with cudaProfilerStart/
+    Stop so an external profiler started with --profile-from-start off records
+    exactly the timed launches."""
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if profile:
+        torch.cuda.cudart().cudaProfilerStart()
+    with torch.cuda.stream(stream):
+        a.record(stream)
+        for _ in range(steps):
+            g.replay()
+        b.record(stream)
+    b.synchronize()
+    if profile:
+        torch.cuda.cudart().cudaProfilerStop()
+    torch.cuda.synchronize()
+    barrier(world)
+    return a.elapsed_time(b) / 1e3
+
+
+def per_shape_numbers(stack, M, stream, reps=20):
+    """Each distinct shape alone: one graph of 8 rotating weight copies x reps."""
+    res = {}
+    seen = {}
+    for i, (l, mi, name, N, K) in enumerate(stack.shapes):
+        if name in seen or name in ("k", "up"):          # k == v, up == gate
+            continue
+        seen[name] = i
+    for name, i in seen.items():
+        (_, _, _, N, K) = stack.shapes[i]
+        idx = [j for j, s in enumerate(stack.shapes) if s[2] == name][:8]
+        x = synth.activations(M, K, seed=5, device="cuda")
+        y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(g, stream=stream):
+                for _ in range(reps):
+                    for j in idx:
+                        pk, sc, ze = stack.q[j]
+                        bq.bq_linear(x, pk, sc, ze, N, stack.bits, stack.group, out=y, stream=stream)
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        b.synchronize()
+        t = a.elapsed_time(b) / 1e3 / (reps * len(idx))
+        byts = linear_bytes(N, K, stack.bits, stack.group, M)
+        res[f"{name} {N}x{K}"] = {"us": round(t * 1e6, 2), "GBps": round(byts / t / 1e9, 1)}
+        del g
+    return res
+
+
+def e2e_numbers(stack, Ms, steps, warmup, world):
+    """Same metric through the C ABI with host buffers: every step copies all
+    activations from pinned host memory to the device and all outputs back."""
+    xs_h, ys_h, xs_d, ys_d = {}, {}, {}, {}
+    h2d = d2h = 0
+    for M in Ms:
+        tot_x = sum(M * K for (_, _, _, N, K) in stack.shapes)
+        tot_y = sum(M * N for (_, _, _, N, K) in stack.shapes)
+        xs_h[M] = torch.empty(tot_x, dtype=torch.bfloat16, pin_memory=True)
+        xs_h[M].copy_(synth.normal((tot_x,), 1.0, seed=900 + M, dtype="bf16"))
+        ys_h[M] = torch.empty(tot_y, dtype=torch.bfloat16, pin_memory=True)
+        xs_d[M] = torch.empty(tot_x, dtype=torch.bfloat16, device="cuda")
+        ys_d[M] = torch.empty(tot_y, dtype=torch.bfloat16, device="cuda")
+        h2d += tot_x * 2
+        d2h += tot_y * 2
+    stream = torch.cuda.Stream()
+
+    def one_step():
+        with torch.cuda.stream(stream):
+            for M in Ms:
+                xs_d[M].copy_(xs_h[M], non_blocking=True)
+                ox = oy = 0
+                for i, (l, mi, name, N, K) in enumerate(stack.shapes):
+                    pk, sc, ze = stack.q[i]
+                    bq.bq_linear(xs_d[M][ox:ox + M * K].view(M, K), pk, sc, ze, N, stack.bits, stack.group,
+                                 out=ys_d[M][oy:oy + M * N].view(M, N), stream=stream)
+                    ox += M * K
+                    oy += M * N
+                ys_h[M].copy_(ys_d[M], non_blocking=True)
+
+    for _ in range(warmup):
+        one_step()
+    stream.synchronize()
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        one_step()
+    b.record(stream)
+    b.synchronize()
+    barrier(world)
+    t = a.elapsed_time(b) / 1e3 / steps
+    return t, h2d, d2h
+
+
+def run_gpu(args, world, rank, local):
+    hbm, bf16, bf16_sus, peak_kind = peaks()
+    bits, group = args.bits, (128 if args.bits == 4 else 64)
+    dist_kind = "t4" if args.bits == 2 else "normal"
+    stack = Stack(args.layers, bits, group, seed_offset=rank * 100000, dist_kind=dist_kind,
+                  quant_time=not args.no_quant)
+    Ms = M_SET
+    xs = {M: [synth.activations(M, K, seed=10000 * M + i + rank * 7, device="cuda")
+              for i, (_, _, _, N, K) in enumerate(stack.shapes)] for M in Ms}
+    ys = {M: [torch.empty((M, N), dtype=torch.bfloat16, device="cuda") for (_, _, _, N, K) in stack.shapes]
+          for M in Ms}
+    stream = torch.cuda.Stream()
+    g = stack.make_graph(Ms, xs, ys, stream)
+    torch.cuda.synchronize()
+
+    with ClockSampler(local) as clk:
+        t_total = time_graph(g, args.steps, args.warmup, stream, world, profile=True)
+    t_step = max_over_ranks(t_total / args.steps, world)
+    clocks = clk.summary()
+
+    # per-M graphs (same kernels) for the breakdown
+    per_m = {}
+    for M in Ms:
+        gm = stack.make_graph((M,), xs, ys, stream)
+        tm = time_graph(gm, max(2, args.steps), 1, stream, world) / max(2, args.steps)
+        tm = max_over_ranks(tm, world)
+        bm = stack.step_bytes((M,))
+        per_m[str(M)] = {"ms": round(tm * 1e3, 4), "GBps": round(bm / tm / 1e9, 1),
+                         "frac_of_measured_hbm": round(bm / tm / 1e9 / hbm, 4),
+                         "tokens_per_s": round(M / tm, 1)}
+        del gm
+    shapes = {str(M): per_shape_numbers(stack, M, stream) for M in Ms} if not args.quick else {}
+
+    step_bytes = stack.step_bytes(Ms)
+    value = world * step_bytes / t_step / 1e9
+    launches_per_step = len(Ms) * len(stack.shapes)
+
+    # end to end through the C ABI with host buffers
+    t_e2e, h2d, d2h = e2e_numbers(stack, Ms, max(1, args.steps // 2), 2, world)
+    t_e2e = max_over_ranks(t_e2e, world)
+
+    achieved = step_bytes / t_step / 1e9   # per-GPU: the GEMV is the only kernel in the step
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(achieved / hbm, 4), "traffic": None,
+                "kernel": "gemv_kernel (decode dequant-GEMV, mma.sync bf16)",
+                "peak_kind": peak_kind + " (copy burst)",
+                "frac_of_nominal_8TBps": round(achieved / 8000.0, 4),
+                "bytes_per_launch_avg": round(step_bytes / launches_per_step),
+                "us_per_launch_avg": round(t_step / launches_per_step * 1e6, 3)}
+
+    extra = {"per_M": per_m, "per_shape": shapes, "quantizer_stack": None}
+    if stack.quant:
+        qz = stack.quant
+        extra["quantizer_stack"] = {"weights": qz["weights"], "ms": round(qz["seconds"] * 1e3, 3),
+                                    "weights_per_s": round(qz["weights_per_s"], 1),
+                                    "GBps": round(qz["GBps"], 1), "frac_of_measured_hbm": round(qz["GBps"] / hbm, 4),
+                                    "launches": qz["launches"]}
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(t_step * 1e3, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": f"bf16 x int{bits} -> fp32 acc", "data": "synthetic",
+        "config": {"workload": f"Llama-3-8B-shaped decode stack, {args.layers} layers x 7 linears, "
+                               f"INT{bits} g{group} weight-only, M in {{1,4,16}} per step",
+                   "layers": args.layers, "bits": bits, "group": group, "M": list(Ms),
+                   "weights": "fp16 N(0,0.02)" if bits == 4 else "fp16 Student-t4 std 0.02 + 0.1% x10 outlier cols",
+                   "activations": "bf16 N(0,1)", "l2": "inputs larger than L2 (packed stack %.2f GB)" %
+                   (sum(weight_bytes(N, K, bits, group) for (_, _, _, N, K) in stack.shapes) / 1e9),
+                   "graph": "one CUDA graph per step", "parallelism": f"replicas x{world} (independent batches)"},
+        "roofline": roofline,
+        "clocks": clocks,
+        "e2e": {"value": round(world * step_bytes / t_e2e / 1e9, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(t_e2e * 1e3, 4)},
+        "gpu_launches": launches_per_step * args.steps,
+        "extra": extra,
+    }
+    return out
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (baseline and reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(threads: int, layers_sample: int = 1, Ms=M_SET, bits=4):
+    """Time the CPU oracle's linear layer on a bounded sample of the stack:
+    the first `layers_sample` layers' 7 linears at every M of the step."""
+    from oracle import oracle as O  # test infrastructure, CPU baseline only
+    group = 128 if bits == 4 else 64
+    shapes = stack_shapes(layers_sample)
+    total_bytes = 0
+    t_lin = 0.0
+    for (l, mi, name, N, K) in shapes:
+        W = synth.normal((N, K), 0.02, synth.weight_seed(l, mi), "f16", "cpu")
+        codes, scales, zeros = O.quantize(synth.bits16(W), "f16", bits, group, threads=threads)
+        for M in Ms:
+            x = O.decode_f64(synth.bits16(synth.activations(M, K, seed=M + mi, device="cpu")), "bf16")
+            t0 = time.perf_counter()
+            O.linear_f64(x, codes, scales, zeros, group, threads=threads)
+            t_lin += time.perf_counter() - t0
+            total_bytes += linear_bytes(N, K, bits, group, M)
+    return total_bytes / t_lin / 1e9, t_lin, total_bytes
+
+
+def cpu_baseline(args):
+    threads = os.cpu_count() or 1
+    gbps, secs, byts = oracle_sample(threads, args.oracle_layers, bits=args.bits)
+    return {"value": round(gbps, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"first {args.oracle_layers} layer(s) x 7 linears x M in {{1,4,16}} "
+                      f"({byts / 1e6:.1f} MB of weight traffic, {secs:.1f} s); fp64 linear over dequantized weights"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    threads = os.cpu_count() or 1
+    for _ in range(args.warmup):
+        pass
+    times, gbps_all = [], []
+    byts_step = None
+    for _ in range(max(1, args.steps)):
+        gbps, secs, byts = oracle_sample(threads, args.oracle_layers, bits=args.bits)
+        times.append(secs)
+        byts_step = byts
+    t = statistics.median(times)
+    value = byts_step / t / 1e9
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t * 1e3, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"Llama-3-8B-shaped decode stack, INT{args.bits}, M in {{1,4,16}} "
+                               f"(bounded sample: first {args.oracle_layers} layer(s))"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": f"first {args.oracle_layers} layer(s) x 7 linears x M in {{1,4,16}} per step"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--bits", type=int, default=4, choices=[2, 4])
+    ap.add_argument("--layers", type=int, default=synth.LLAMA3_8B_LAYERS)
+    ap.add_argument("--oracle-layers", type=int, default=1)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-quant", action="store_true")
+    ap.add_argument("--quick", action="store_true", help="skip the per-shape breakdown")
+    args = ap.parse_args()
+
+    world, rank, local = dist_setup()
+    if args.gpus != world and world > 1:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    if args.warmup < 3:
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+
+    if args.impl == "reference":
+        out = run_reference(args, world, rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+    else:
+        if not torch.cuda.is_available():
+            raise SystemExit("bench.py: a CUDA GPU is required for the GPU arm")
+        bq.lib()  # fail loudly if the CUDA library is missing
+        out = run_gpu(args, world, rank, local)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                out["cpu_baseline"] = cpu_baseline(args)
+            print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

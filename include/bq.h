@@ -1,0 +1,191 @@
+/*
+ * bq.h -- C ABI of the B200 (sm_100a) group-wise MinMax weight quantizer and
+ * weight-only linear layer.
+ *
+ * The method (GreenBitAI article "只需单卡 RTX 3090，低比特量化训练就能实现
+ * LLaMA-3 8B 全参微调", paragraph on the quantizer): classic Group-wise MinMax
+ * quantization, used only as INT4 with group size 128 and INT2 with group
+ * size 64, mixed per layer (Layer-mix) or per output-channel block
+ * (Channel-mix).  Per group of `group` consecutive weights of one row
+ * ("大模型量化实战：从原理到4-bit部署的完整指南", section 2.2; "低比特量化 /
+ * Low-bit Quantization", sections "Group Quantization" and "Zero Point"):
+ *
+ *     lo = min(min x, 0)     hi = max(max x, 0)          (range widened to 0)
+ *     s  = (hi - lo) / (2^b - 1)                          fp32, round to nearest even
+ *     z  = round(-lo / s)                                 half to even, 0 <= z <= 2^b-1
+ *     q  = clamp(round(x / s) + z, 0, 2^b - 1)            x/s one fp32 division
+ *     dequant(q) = (q - z) * s
+ *     an all-zero group stores s = 0, z = 0, q = 0
+ *
+ * and the weight-only linear layer y = x . dequant(W)^T (survey "A Survey of
+ * Low-bit Large Language Models", section 6.2 weight-only: dequantize, then a
+ * 16-bit matmul; "大模型量化实战" section 3.3: dequantize and multiply in one
+ * fused kernel).  No dequantized weight is ever written by the linear layer.
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ *  - W is [rows, cols] row-major: rows = N = output channels, cols = K = input
+ *    channels.  Groups run along cols inside one row.
+ *  - Every buffer pointer is a DEVICE pointer unless the argument says "host".
+ *    The caller owns and allocates every buffer; the library never allocates
+ *    or frees memory.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Work is enqueued asynchronously; argument errors are returned
+ *    synchronously before anything is enqueued.
+ *  - Pointers to W, x, y, packed codes and dequantized output must be 16-byte
+ *    aligned; scales and zeros 4-byte and 1-byte aligned.
+ *  - Conditions only the device can see (a non-finite weight, a wait that
+ *    gave up) set a device status word; read it with bq_device_status().
+ *  - On a CUDA launch failure the entry point returns BQ_ERR_CUDA.
+ */
+#ifndef BQ_H
+#define BQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BQ_OK = 0,
+    BQ_ERR_NULL = 1,        /* a required pointer is NULL */
+    BQ_ERR_SHAPE = 2,       /* sizes are inconsistent or not multiples of a tile */
+    BQ_ERR_ALIGN = 3,       /* a pointer is not aligned as required */
+    BQ_ERR_UNSUPPORTED = 4, /* bits / group / layout / dtype combination not supported */
+    BQ_ERR_WORKSPACE = 5,   /* reserved */
+    BQ_ERR_NONFINITE = 6,   /* device: a weight is NaN/Inf, or a group's fp32 scale overflows */
+    BQ_ERR_TIMEOUT = 7,     /* device: a bounded wait inside a kernel gave up */
+    BQ_ERR_CUDA = 8         /* a CUDA runtime call or launch failed */
+} bq_status;
+
+typedef enum { BQ_F16 = 0, BQ_BF16 = 1, BQ_F32 = 2 } bq_dtype;
+
+/*
+ * Packed-code layouts.  Both hold b-bit codes, b in {2, 4}; a matrix takes
+ * rows * cols * b / 8 bytes in either layout.
+ *
+ * BQ_LAYOUT_CANONICAL: row-major; code k of a row is field k mod (32/b) of
+ *   little-endian 32-bit word k / (32/b) of that row, fields numbered from the
+ *   least significant bit.  Needs cols * b % 32 == 0.
+ *
+ * BQ_LAYOUT_INTERLEAVED: the layout the linear kernels read.  The matrix is
+ *   cut into 512-byte tiles of 16 rows by T columns (T = 64 for 4-bit, 128 for
+ *   2-bit), stored row-block major (tile (rb, kt) at 512 * (rb * cols/T + kt)).
+ *   Inside a tile, 16-byte "lane" L (0..31) serves rows r = L/4 and r + 8 and,
+ *   in every run of 16 columns, the column pairs (2c, 2c+1) and (2c+8, 2c+9),
+ *   c = L % 4.  Slot i of a run is (row r, low pair), (row r+8, low pair),
+ *   (row r, high pair), (row r+8, high pair) for i = 0..3.
+ *     4-bit: 32-bit word j of the lane holds run j; slot i keeps its even
+ *            column in nibble i and its odd column in nibble i + 4.
+ *     2-bit: word j holds runs 2j (fields 0..3, 8..11) and 2j+1 (fields
+ *            4..7, 12..15); slot i of run 2j+h keeps its even column in field
+ *            4h + i and its odd column in field 4h + i + 8.
+ *   Needs rows % 16 == 0 and cols % T == 0.  With this order a lane's 16-byte
+ *   load is already in the register order of a 16x8x16 bf16 tensor-core
+ *   fragment, and one AND/OR with a magic exponent turns two codes into a
+ *   bf16x2 pair.
+ */
+typedef enum { BQ_LAYOUT_CANONICAL = 0, BQ_LAYOUT_INTERLEAVED = 1 } bq_layout;
+
+/* Bytes of packed codes for a rows x cols matrix at `bits` (no metadata). */
+size_t bq_packed_bytes(int64_t rows, int64_t cols, int bits);
+
+/* Number of groups (= number of scales = number of zeros). */
+size_t bq_group_count(int64_t rows, int64_t cols, int group);
+
+/*
+ * Mixed precision (Layer-mix / Channel-mix, GreenBitAI article, paragraph on
+ * the mixed-precision search space).  A bit map assigns one width to every
+ * block of 128 consecutive rows: 4 (group 128) or 2 (group 64).  Layer-mix
+ * is the special case of one width per matrix.  A mixed matrix stores its
+ * blocks one after the other in row order: block i's packed codes start at
+ * byte code_off[i] and its scales / zeros at element group_off[i], each
+ * block laid out as an independent 128 x cols matrix.
+ *
+ * bq_mixed_offsets: host-side helper.  bit_map (host, rows/128 entries);
+ * code_off and group_off (host, rows/128 + 1 entries each) receive the
+ * running sums; the last entries are the totals.  Needs rows % 128 == 0.
+ */
+bq_status bq_mixed_offsets(const uint8_t *bit_map, int64_t rows, int64_t cols,
+                           int64_t *code_off, int64_t *group_off);
+
+/*
+ * bq_quantize: quantize W and pack the codes.
+ *   W        [rows, cols] of wtype (BQ_F16 or BQ_BF16), 16-byte aligned
+ *   bits     4 or 2
+ *   group    production: 128 with bits 4, 64 with bits 2.  Also accepted for
+ *            tests: any of 16, 32, 64, 128, 256 dividing cols (canonical layout
+ *            also 8).
+ *   layout   BQ_LAYOUT_CANONICAL or BQ_LAYOUT_INTERLEAVED (shape rules above)
+ *   packed   [bq_packed_bytes(rows, cols, bits)] bytes, 16-byte aligned
+ *   scales   [rows, cols/group] fp32
+ *   zeros    [rows, cols/group] uint8
+ * A non-finite weight, or a group whose scale overflows fp32, sets
+ * BQ_ERR_NONFINITE in the device status word; that group's outputs are then
+ * unspecified.
+ */
+bq_status bq_quantize(const void *W, bq_dtype wtype, int64_t rows, int64_t cols,
+                      int bits, int group, bq_layout layout,
+                      void *packed, float *scales, uint8_t *zeros, void *stream);
+
+/*
+ * bq_quantize_mixed: quantize with a per-128-row-block width.
+ *   bit_map  DEVICE array of rows/128 bytes, each 4 or 2 (any other value sets
+ *            BQ_ERR_UNSUPPORTED in the device status word and skips the block)
+ *   packed / scales / zeros: sized by the totals of bq_mixed_offsets(); the
+ *            device computes each block's offsets from bit_map itself.
+ */
+bq_status bq_quantize_mixed(const void *W, bq_dtype wtype, int64_t rows, int64_t cols,
+                            const uint8_t *bit_map, bq_layout layout,
+                            void *packed, float *scales, uint8_t *zeros, void *stream);
+
+/*
+ * bq_dequantize: W_out[rows, cols] = (q - z) * s, computed in fp32 and
+ * rounded once to otype (BQ_F32, BQ_F16 or BQ_BF16).  A test / inspection
+ * utility; the linear layer never calls it.
+ *   bit_map  NULL for a uniform matrix (bits, group used), else a DEVICE
+ *            bit map as in bq_quantize_mixed (bits and group ignored).
+ */
+bq_status bq_dequantize(const void *packed, const float *scales, const uint8_t *zeros,
+                        const uint8_t *bit_map, int bits, int group,
+                        int64_t rows, int64_t cols, bq_layout layout,
+                        void *W_out, bq_dtype otype, void *stream);
+
+/*
+ * bq_linear: y[M, N] = x[M, K] . dequant(W)^T.
+ *   x        [M, K] of xtype (BQ_BF16 or BQ_F16), 16-byte aligned rows (K % 8 == 0)
+ *   packed / scales / zeros: from bq_quantize in BQ_LAYOUT_INTERLEAVED
+ *   bit_map  NULL for a uniform matrix (bits, group used; production pairs
+ *            (4, 128) and (2, 64), tests also group 32 and 256), else a DEVICE
+ *            bit map as in bq_quantize_mixed (bits, group ignored)
+ *   y        [M, N] of xtype, written in full
+ * Products are accumulated in fp32 per group on exact (q - z) operands, then
+ * scaled by the group's fp32 s and summed in fp32; y is rounded once.
+ * M <= 16 runs the decode kernel (split-K dequant-GEMV on tensor cores);
+ * larger M runs the prefill kernel.  Needs N % 16 == 0 (N % 128 == 0 with a
+ * bit map) and K a multiple of the tile width of every width used.
+ */
+bq_status bq_linear(const void *x, bq_dtype xtype, int64_t M, int64_t K,
+                    const void *packed, const float *scales, const uint8_t *zeros,
+                    const uint8_t *bit_map, int bits, int group, int64_t N,
+                    bq_layout layout, void *y, void *stream);
+
+/*
+ * bq_device_status: synchronize `stream`, return the first error recorded by
+ * a kernel since the last call (BQ_OK if none) and clear it.
+ */
+bq_status bq_device_status(void *stream);
+
+/* Human-readable name of a status code (static string). */
+const char *bq_status_string(bq_status status);
+
+/* Library version string, for logs. */
+const char *bq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BQ_H */

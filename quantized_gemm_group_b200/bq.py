@@ -1,0 +1,211 @@
+"""Thin Python binding of the C ABI in ``include/bq.h`` (``libbq.so``).
+
+Argument marshalling only: every step of the quantizer and the linear layer
+runs in the library's CUDA kernels.  Tensors are torch CUDA tensors used as
+plain device buffers; outputs are allocated here with torch and their
+pointers passed down.  There is no fallback: if the library is missing or a
+call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+from . import build as _build
+
+LIB_PATH = _build.LIB
+
+# enums, mirrored from include/bq.h
+BQ_OK, BQ_ERR_NULL, BQ_ERR_SHAPE, BQ_ERR_ALIGN, BQ_ERR_UNSUPPORTED = 0, 1, 2, 3, 4
+BQ_ERR_WORKSPACE, BQ_ERR_NONFINITE, BQ_ERR_TIMEOUT, BQ_ERR_CUDA = 5, 6, 7, 8
+BQ_F16, BQ_BF16, BQ_F32 = 0, 1, 2
+BQ_LAYOUT_CANONICAL, BQ_LAYOUT_INTERLEAVED = 0, 1
+
+LAYOUTS = {"canonical": BQ_LAYOUT_CANONICAL, "interleaved": BQ_LAYOUT_INTERLEAVED}
+DTYPE_CODE = {torch.float16: BQ_F16, torch.bfloat16: BQ_BF16, torch.float32: BQ_F32}
+CODE_DTYPE = {v: k for k, v in DTYPE_CODE.items()}
+GROUP_OF_BITS = {4: 128, 2: 64}
+
+#: every symbol include/bq.h declares
+EXPORTS = (
+    "bq_packed_bytes", "bq_group_count", "bq_mixed_offsets", "bq_quantize", "bq_quantize_mixed",
+    "bq_dequantize", "bq_linear", "bq_device_status", "bq_status_string", "bq_version",
+)
+
+
+class BQError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn}: {status_string(status)}")
+
+
+_lib = None
+
+
+def lib(path: str | None = None):
+    """Load libbq.so (raises if it is missing; build it with build.build())."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise FileNotFoundError(f"{p} is missing: build the CUDA library first "
+                                "(python -m quantized_gemm_group_b200.build)")
+    L = ctypes.CDLL(p)
+    i64, i32, vp, u8p = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p
+    L.bq_packed_bytes.argtypes = [i64, i64, i32]
+    L.bq_packed_bytes.restype = ctypes.c_size_t
+    L.bq_group_count.argtypes = [i64, i64, i32]
+    L.bq_group_count.restype = ctypes.c_size_t
+    L.bq_mixed_offsets.argtypes = [u8p, i64, i64, vp, vp]
+    L.bq_mixed_offsets.restype = i32
+    L.bq_quantize.argtypes = [vp, i32, i64, i64, i32, i32, i32, vp, vp, vp, vp]
+    L.bq_quantize.restype = i32
+    L.bq_quantize_mixed.argtypes = [vp, i32, i64, i64, vp, i32, vp, vp, vp, vp]
+    L.bq_quantize_mixed.restype = i32
+    L.bq_dequantize.argtypes = [vp, vp, vp, vp, i32, i32, i64, i64, i32, vp, i32, vp]
+    L.bq_dequantize.restype = i32
+    L.bq_linear.argtypes = [vp, i32, i64, i64, vp, vp, vp, vp, i32, i32, i64, i32, vp, vp]
+    L.bq_linear.restype = i32
+    L.bq_device_status.argtypes = [vp]
+    L.bq_device_status.restype = i32
+    L.bq_status_string.argtypes = [i32]
+    L.bq_status_string.restype = ctypes.c_char_p
+    L.bq_version.argtypes = []
+    L.bq_version.restype = ctypes.c_char_p
+    if path is None:
+        _lib = L
+    return L
+
+
+def status_string(status: int) -> str:
+    return lib().bq_status_string(int(status)).decode()
+
+
+def _check(fn: str, status: int):
+    if status != BQ_OK:
+        raise BQError(fn, status)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+# ---------------------------------------------------------------------------
+# size queries
+# ---------------------------------------------------------------------------
+
+def bq_packed_bytes(rows: int, cols: int, bits: int) -> int:
+    return int(lib().bq_packed_bytes(rows, cols, bits))
+
+
+def bq_group_count(rows: int, cols: int, group: int) -> int:
+    return int(lib().bq_group_count(rows, cols, group))
+
+
+def bq_mixed_offsets(bit_map, rows: int, cols: int):
+    bm = np.ascontiguousarray(np.asarray(bit_map, dtype=np.uint8))
+    nb = rows // 128
+    co = np.zeros(nb + 1, dtype=np.int64)
+    go = np.zeros(nb + 1, dtype=np.int64)
+    _check("bq_mixed_offsets", lib().bq_mixed_offsets(bm.ctypes.data_as(ctypes.c_void_p), rows, cols,
+                                                      co.ctypes.data_as(ctypes.c_void_p),
+                                                      go.ctypes.data_as(ctypes.c_void_p)))
+    return co, go
+
+
+# ---------------------------------------------------------------------------
+# quantize / dequantize / linear
+# ---------------------------------------------------------------------------
+
+def bq_quantize(W: torch.Tensor, bits: int, group: int | None = None, layout: str = "interleaved",
+                out=None, stream=None):
+    """Quantize W [N, K] (fp16/bf16, CUDA).  Returns (packed u8, scales f32 [N, K/g], zeros u8 [N, K/g])."""
+    group = group or GROUP_OF_BITS[bits]
+    N, K = W.shape
+    if out is None:
+        packed = torch.empty(max(1, bq_packed_bytes(N, K, bits)), dtype=torch.uint8, device=W.device)
+        scales = torch.empty((N, K // group), dtype=torch.float32, device=W.device)
+        zeros = torch.empty((N, K // group), dtype=torch.uint8, device=W.device)
+    else:
+        packed, scales, zeros = out
+    st = lib().bq_quantize(_ptr(W), DTYPE_CODE[W.dtype], N, K, bits, group, LAYOUTS[layout],
+                           _ptr(packed), _ptr(scales), _ptr(zeros), _stream(stream))
+    _check("bq_quantize", st)
+    return packed, scales, zeros
+
+
+def mixed_sizes(bit_map, rows: int, cols: int):
+    co, go = bq_mixed_offsets(bit_map, rows, cols)
+    return int(co[-1]), int(go[-1])
+
+
+def bq_quantize_mixed(W: torch.Tensor, bit_map, layout: str = "interleaved", stream=None):
+    """Per-128-row-block width (4 -> group 128, 2 -> group 64).  bit_map: host sequence.
+    Returns (packed, scales, zeros, bit_map_dev)."""
+    N, K = W.shape
+    code_bytes, groups = mixed_sizes(bit_map, N, K)
+    bm = torch.as_tensor(np.asarray(bit_map, dtype=np.uint8)).to(W.device)
+    packed = torch.empty(max(1, code_bytes), dtype=torch.uint8, device=W.device)
+    scales = torch.empty(max(1, groups), dtype=torch.float32, device=W.device)
+    zeros = torch.empty(max(1, groups), dtype=torch.uint8, device=W.device)
+    st = lib().bq_quantize_mixed(_ptr(W), DTYPE_CODE[W.dtype], N, K, _ptr(bm), LAYOUTS[layout],
+                                 _ptr(packed), _ptr(scales), _ptr(zeros), _stream(stream))
+    _check("bq_quantize_mixed", st)
+    return packed, scales, zeros, bm
+
+
+def bq_dequantize(packed, scales, zeros, rows: int, cols: int, bits: int = 4, group: int | None = None,
+                  layout: str = "interleaved", out_dtype=torch.float32, bit_map_dev=None, stream=None):
+    group = group or GROUP_OF_BITS.get(bits, 0)
+    out = torch.empty((rows, cols), dtype=out_dtype, device=packed.device)
+    st = lib().bq_dequantize(_ptr(packed), _ptr(scales), _ptr(zeros), _ptr(bit_map_dev), bits, group,
+                             rows, cols, LAYOUTS[layout], _ptr(out), DTYPE_CODE[out_dtype], _stream(stream))
+    _check("bq_dequantize", st)
+    return out
+
+
+def bq_linear(x: torch.Tensor, packed, scales, zeros, N: int, bits: int = 4, group: int | None = None,
+              bit_map_dev=None, layout: str = "interleaved", out=None, stream=None):
+    """y [M, N] = x [M, K] . dequant(W)^T, y in x's dtype."""
+    group = group or GROUP_OF_BITS.get(bits, 0)
+    M, K = x.shape
+    y = out if out is not None else torch.empty((M, N), dtype=x.dtype, device=x.device)
+    st = lib().bq_linear(_ptr(x), DTYPE_CODE[x.dtype], M, K, _ptr(packed), _ptr(scales), _ptr(zeros),
+                         _ptr(bit_map_dev), bits, group, N, LAYOUTS[layout], _ptr(y), _stream(stream))
+    _check("bq_linear", st)
+    return y
+
+
+def bq_device_status(stream=None) -> int:
+    return int(lib().bq_device_status(_stream(stream)))
+
+
+def bq_version() -> str:
+    return lib().bq_version().decode()
+
+
+# ---------------------------------------------------------------------------
+# host-buffer path (end-to-end: pinned host in, host out, through the C ABI)
+# ---------------------------------------------------------------------------
+
+def bq_linear_host(x_host: torch.Tensor, packed, scales, zeros, N: int, bits: int = 4, group=None,
+                   bit_map_dev=None, x_dev=None, y_dev=None, y_host=None, stream=None):
+    """Copy x from (pinned) host memory, run bq_linear, copy y back to host."""
+    s = stream or torch.cuda.current_stream()
+    if x_dev is None:
+        x_dev = torch.empty(x_host.shape, dtype=x_host.dtype, device="cuda")
+    x_dev.copy_(x_host, non_blocking=True)
+    y_dev = bq_linear(x_dev, packed, scales, zeros, N, bits, group, bit_map_dev, out=y_dev, stream=s)
+    if y_host is None:
+        y_host = torch.empty(y_dev.shape, dtype=y_dev.dtype, pin_memory=True)
+    y_host.copy_(y_dev, non_blocking=True)
+    return y_host

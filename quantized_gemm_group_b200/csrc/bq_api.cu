@@ -1,0 +1,447 @@
+// bq_api.cu -- C ABI of the quantizer / weight-only linear library (see
+// include/bq.h for the contract of every entry point).  Host-side argument
+// validation, launch geometry and dispatch onto the sm_100a kernels.
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/bq.h"
+#include "common.cuh"
+#include "dequant.cuh"
+#include "gemv.cuh"
+#include "quantize.cuh"
+
+using namespace bq;
+
+namespace {
+
+constexpr int kThreads = 256;
+
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return 148;
+  if (!cached[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bq_status launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+}
+
+int64_t grid_for(int64_t warps_of_work) {
+  int64_t blocks = (warps_of_work + (kThreads / 32) - 1) / (kThreads / 32);
+  int64_t cap = (int64_t)sm_count() * 8;  // 8 x 256 threads = 2048 per SM
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  return blocks;
+}
+
+bool valid_bits(int bits) { return bits == 2 || bits == 4; }
+int tile_width(int bits) { return bits == 4 ? 64 : 128; }
+
+// ---------------------------------------------------------------------------
+// quantize dispatch
+// ---------------------------------------------------------------------------
+
+template <int WT, int BITS>
+bq_status quantize_canonical(const uint16_t *W, int64_t elems, int group, uint8_t *packed, float *scales,
+                             uint8_t *zeros, cudaStream_t st) {
+  const int64_t grid = grid_for((elems + 255) / 256);
+#define BQ_QC(G)                                                                              \
+  case G:                                                                                     \
+    quantize_canonical_kernel<WT, BITS, G, 4><<<grid, kThreads, 0, st>>>(W, elems, packed, scales, zeros); \
+    break;
+  switch (group) {
+    BQ_QC(8) BQ_QC(16) BQ_QC(32) BQ_QC(64) BQ_QC(128) BQ_QC(256)
+    default: return BQ_ERR_UNSUPPORTED;
+  }
+#undef BQ_QC
+  return launch_status();
+}
+
+template <int WT, int BITS>
+bq_status quantize_tiled(const uint16_t *W, int64_t N, int64_t K, int group, uint8_t *packed, float *scales,
+                         uint8_t *zeros, cudaStream_t st) {
+  const int64_t U = group > tile_width(BITS) ? group : tile_width(BITS);
+  const int64_t grid = grid_for((N / 16) * (K / U));
+#define BQ_QT(G)                                                                           \
+  case G:                                                                                  \
+    quantize_tiled_kernel<WT, BITS, G><<<grid, kThreads, 0, st>>>(W, N, K, packed, scales, zeros); \
+    break;
+  switch (group) {
+    BQ_QT(16) BQ_QT(32) BQ_QT(64) BQ_QT(128) BQ_QT(256)
+    default: return BQ_ERR_UNSUPPORTED;
+  }
+#undef BQ_QT
+  return launch_status();
+}
+
+bool canonical_group_ok(int g) { return g == 8 || g == 16 || g == 32 || g == 64 || g == 128 || g == 256; }
+bool tiled_group_ok(int g) { return g == 16 || g == 32 || g == 64 || g == 128 || g == 256; }
+
+// ---------------------------------------------------------------------------
+// dequant dispatch
+// ---------------------------------------------------------------------------
+
+template <int OT>
+bq_status dequant_uniform(const uint8_t *packed, const float *scales, const uint8_t *zeros, int bits, int group,
+                          int64_t N, int64_t K, bq_layout layout, void *out, cudaStream_t st) {
+  using T = typename OutT<OT>::T;
+  T *o = reinterpret_cast<T *>(out);
+  if (layout == BQ_LAYOUT_CANONICAL) {
+    const int64_t elems = N * K;
+    const int64_t grid = grid_for((elems / 8 + 31) / 32);
+    if (bits == 4) dequant_canonical_kernel<OT, 4><<<grid, kThreads, 0, st>>>(packed, scales, zeros, group, elems, o);
+    else dequant_canonical_kernel<OT, 2><<<grid, kThreads, 0, st>>>(packed, scales, zeros, group, elems, o);
+  } else {
+    const int64_t tiles = (N / 16) * (K / tile_width(bits));
+    const int64_t grid = grid_for(tiles);
+    if (bits == 4) dequant_tiled_kernel<OT, 4><<<grid, kThreads, 0, st>>>(packed, scales, zeros, group, N, K, o);
+    else dequant_tiled_kernel<OT, 2><<<grid, kThreads, 0, st>>>(packed, scales, zeros, group, N, K, o);
+  }
+  return launch_status();
+}
+
+template <int OT>
+bq_status dequant_mixed(const uint8_t *packed, const float *scales, const uint8_t *zeros, const uint8_t *bit_map,
+                        int64_t N, int64_t K, bq_layout layout, void *out, cudaStream_t st) {
+  using T = typename OutT<OT>::T;
+  const int64_t grid = grid_for(N / 128);
+  if (layout == BQ_LAYOUT_CANONICAL)
+    dequant_mixed_kernel<OT, false><<<grid, kThreads, 0, st>>>(packed, scales, zeros, bit_map, N, K, reinterpret_cast<T *>(out));
+  else
+    dequant_mixed_kernel<OT, true><<<grid, kThreads, 0, st>>>(packed, scales, zeros, bit_map, N, K, reinterpret_cast<T *>(out));
+  return launch_status();
+}
+
+// ---------------------------------------------------------------------------
+// GEMV (M <= 16) geometry and dispatch
+// ---------------------------------------------------------------------------
+
+struct Geom {
+  int NB, R, NWR, NWK, S;
+  int64_t KC, KW;
+};
+
+bool pdl_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char *e = getenv("BQ_PDL");
+    v = (e && e[0] == '1') ? 1 : 0;
+  }
+  return v == 1;
+}
+
+Geom gemv_geometry(int M, int64_t N, int64_t K, int64_t SU, bool mixed) {
+  Geom g;
+  g.NB = (M <= 8) ? 1 : 2;
+  g.R = (N % 32 == 0) ? 2 : 1;
+  g.NWR = 1;
+  for (int c : {4, 2, 1}) {
+    if (N % (16 * g.R * c) == 0) { g.NWR = c; break; }
+  }
+  if (mixed) { g.R = 2; g.NWR = 4; }
+  const int64_t rows = 16 * g.R * g.NWR;
+  const int64_t row_ctas = N / rows;
+  const int64_t units = K / SU;
+  const int64_t target_warps = (int64_t)sm_count() * 14;
+  const int max_nwk = 8 / g.NWR;
+  // smallest split d = S * NWK (S <= 8 CTAs per cluster, NWK <= max_nwk
+  // warps along K) dividing the units that reaches the target warp count
+  int best_s = 1, best_nwk = 1;
+  for (int d = 1; d <= 8 * max_nwk; ++d) {
+    if (units % d) continue;
+    int nwk = 0;
+    for (int c = 1; c <= max_nwk; ++c) {
+      if (d % c == 0 && d / c <= 8) { nwk = c; break; }
+    }
+    if (!nwk) continue;
+    best_s = d / nwk;
+    best_nwk = nwk;
+    if (row_ctas * g.NWR * d >= target_warps) break;
+  }
+  g.NWK = best_nwk;
+  g.S = best_s;
+  g.KC = K / g.S;
+  g.KW = g.KC / g.NWK;
+  return g;
+}
+
+template <int XT, int BITS, int G, int NB, int R, bool MIXED>
+bq_status launch_gemv_t(const Geom &g, const uint16_t *x, int M, int64_t K, const uint8_t *packed,
+                        const float *scales, const uint8_t *zeros, const uint8_t *bit_map, int64_t N,
+                        uint16_t *y, cudaStream_t st) {
+  auto kern = gemv_kernel<XT, BITS, G, NB, R, MIXED>;
+  const size_t smem = gemv_smem_bytes(NB, R, g.NWR, g.NWK, g.KC);
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
+      return BQ_ERR_CUDA;
+    attr_set = true;
+  }
+  if (smem > 227 * 1024) return BQ_ERR_SHAPE;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(N / (16 * R * g.NWR)), (unsigned)g.S, 1);
+  cfg.blockDim = dim3((unsigned)(32 * g.NWR * g.NWK), 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attrs[2];
+  int na = 0;
+  attrs[na].id = cudaLaunchAttributeClusterDimension;
+  attrs[na].val.clusterDim.x = 1;
+  attrs[na].val.clusterDim.y = (unsigned)g.S;
+  attrs[na].val.clusterDim.z = 1;
+  ++na;
+  if (pdl_enabled()) {
+    attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attrs[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  cfg.attrs = attrs;
+  cfg.numAttrs = na;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, x, M, K, packed, scales, zeros, bit_map, N, y, g.KC, g.KW, g.NWR);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return BQ_ERR_CUDA;
+  }
+  return BQ_OK;
+}
+
+template <int XT, int BITS, int G, bool MIXED>
+bq_status launch_gemv_nb(const Geom &g, const uint16_t *x, int M, int64_t K, const uint8_t *packed,
+                         const float *scales, const uint8_t *zeros, const uint8_t *bit_map, int64_t N,
+                         uint16_t *y, cudaStream_t st) {
+  if (g.NB == 1) {
+    if (g.R == 2) return launch_gemv_t<XT, BITS, G, 1, 2, MIXED>(g, x, M, K, packed, scales, zeros, bit_map, N, y, st);
+    return launch_gemv_t<XT, BITS, G, 1, 1, MIXED>(g, x, M, K, packed, scales, zeros, bit_map, N, y, st);
+  }
+  if (g.R == 2) return launch_gemv_t<XT, BITS, G, 2, 2, MIXED>(g, x, M, K, packed, scales, zeros, bit_map, N, y, st);
+  return launch_gemv_t<XT, BITS, G, 2, 1, MIXED>(g, x, M, K, packed, scales, zeros, bit_map, N, y, st);
+}
+
+template <int XT>
+bq_status gemv_dispatch(const uint16_t *x, int M, int64_t K, const uint8_t *packed, const float *scales,
+                        const uint8_t *zeros, const uint8_t *bit_map, int bits, int group, int64_t N, uint16_t *y,
+                        cudaStream_t st) {
+  if (bit_map) {
+    Geom g = gemv_geometry(M, N, K, 128, true);
+    return launch_gemv_nb<XT, 4, 128, true>(g, x, M, K, packed, scales, zeros, bit_map, N, y, st);
+  }
+  const int64_t SU = group > tile_width(bits) ? group : tile_width(bits);
+  Geom g = gemv_geometry(M, N, K, SU, false);
+#define BQ_GV(B, G_)                                                                                 \
+  if (bits == B && group == G_)                                                                      \
+    return launch_gemv_nb<XT, B, G_, false>(g, x, M, K, packed, scales, zeros, nullptr, N, y, st);
+  BQ_GV(4, 128) BQ_GV(2, 64) BQ_GV(4, 32) BQ_GV(4, 64) BQ_GV(4, 256) BQ_GV(2, 32) BQ_GV(2, 128) BQ_GV(2, 256)
+#undef BQ_GV
+  return BQ_ERR_UNSUPPORTED;
+}
+
+bool linear_group_ok(int bits, int g) {
+  (void)bits;
+  return g == 32 || g == 64 || g == 128 || g == 256;
+}
+
+}  // namespace
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+
+extern "C" {
+
+const char *bq_version(void) { return "bq 0.1 (sm_100a)"; }
+
+const char *bq_status_string(bq_status s) {
+  switch (s) {
+    case BQ_OK: return "BQ_OK";
+    case BQ_ERR_NULL: return "BQ_ERR_NULL: a required pointer is NULL";
+    case BQ_ERR_SHAPE: return "BQ_ERR_SHAPE: sizes inconsistent or not tile multiples";
+    case BQ_ERR_ALIGN: return "BQ_ERR_ALIGN: pointer not aligned as required";
+    case BQ_ERR_UNSUPPORTED: return "BQ_ERR_UNSUPPORTED: bits/group/layout/dtype not supported";
+    case BQ_ERR_WORKSPACE: return "BQ_ERR_WORKSPACE";
+    case BQ_ERR_NONFINITE: return "BQ_ERR_NONFINITE: non-finite weight or overflowing scale";
+    case BQ_ERR_TIMEOUT: return "BQ_ERR_TIMEOUT: a bounded wait in a kernel gave up";
+    case BQ_ERR_CUDA: return "BQ_ERR_CUDA: CUDA runtime error";
+  }
+  return "unknown bq_status";
+}
+
+size_t bq_packed_bytes(int64_t rows, int64_t cols, int bits) {
+  if (rows < 0 || cols < 0 || !valid_bits(bits)) return 0;
+  return (size_t)(rows * cols * bits / 8);
+}
+
+size_t bq_group_count(int64_t rows, int64_t cols, int group) {
+  if (rows < 0 || cols < 0 || group <= 0 || cols % group) return 0;
+  return (size_t)(rows * (cols / group));
+}
+
+bq_status bq_mixed_offsets(const uint8_t *bit_map, int64_t rows, int64_t cols, int64_t *code_off,
+                           int64_t *group_off) {
+  if (!bit_map || !code_off || !group_off) return BQ_ERR_NULL;
+  if (rows < 0 || cols < 0 || rows % 128) return BQ_ERR_SHAPE;
+  const int64_t nb = rows / 128;
+  code_off[0] = 0;
+  group_off[0] = 0;
+  for (int64_t i = 0; i < nb; ++i) {
+    const int b = bit_map[i];
+    if (!valid_bits(b)) return BQ_ERR_UNSUPPORTED;
+    const int g = (b == 4) ? 128 : 64;
+    if (cols % g) return BQ_ERR_SHAPE;
+    code_off[i + 1] = code_off[i] + 128 * cols * b / 8;
+    group_off[i + 1] = group_off[i] + 128 * (cols / g);
+  }
+  return BQ_OK;
+}
+
+bq_status bq_quantize(const void *W, bq_dtype wtype, int64_t rows, int64_t cols, int bits, int group,
+                      bq_layout layout, void *packed, float *scales, uint8_t *zeros, void *stream) {
+  if (rows < 0 || cols < 0) return BQ_ERR_SHAPE;
+  if (!valid_bits(bits) || (wtype != BQ_F16 && wtype != BQ_BF16)) return BQ_ERR_UNSUPPORTED;
+  if (layout != BQ_LAYOUT_CANONICAL && layout != BQ_LAYOUT_INTERLEAVED) return BQ_ERR_UNSUPPORTED;
+  if (layout == BQ_LAYOUT_CANONICAL ? !canonical_group_ok(group) : !tiled_group_ok(group)) return BQ_ERR_UNSUPPORTED;
+  if (cols % group) return BQ_ERR_SHAPE;
+  if (layout == BQ_LAYOUT_CANONICAL) {
+    if ((cols * bits) % 32) return BQ_ERR_SHAPE;
+  } else {
+    const int64_t U = group > tile_width(bits) ? group : tile_width(bits);
+    if (rows % 16 || cols % U) return BQ_ERR_SHAPE;
+  }
+  if (rows == 0 || cols == 0) return BQ_OK;
+  if (!W || !packed || !scales || !zeros) return BQ_ERR_NULL;
+  if (!aligned(W, 16) || !aligned(packed, 16) || !aligned(scales, 4)) return BQ_ERR_ALIGN;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const uint16_t *w = reinterpret_cast<const uint16_t *>(W);
+  uint8_t *pk = reinterpret_cast<uint8_t *>(packed);
+  if (layout == BQ_LAYOUT_CANONICAL) {
+    const int64_t elems = rows * cols;
+    if (wtype == BQ_F16) return bits == 4 ? quantize_canonical<0, 4>(w, elems, group, pk, scales, zeros, st)
+                                          : quantize_canonical<0, 2>(w, elems, group, pk, scales, zeros, st);
+    return bits == 4 ? quantize_canonical<1, 4>(w, elems, group, pk, scales, zeros, st)
+                     : quantize_canonical<1, 2>(w, elems, group, pk, scales, zeros, st);
+  }
+  if (wtype == BQ_F16) return bits == 4 ? quantize_tiled<0, 4>(w, rows, cols, group, pk, scales, zeros, st)
+                                        : quantize_tiled<0, 2>(w, rows, cols, group, pk, scales, zeros, st);
+  return bits == 4 ? quantize_tiled<1, 4>(w, rows, cols, group, pk, scales, zeros, st)
+                   : quantize_tiled<1, 2>(w, rows, cols, group, pk, scales, zeros, st);
+}
+
+bq_status bq_quantize_mixed(const void *W, bq_dtype wtype, int64_t rows, int64_t cols, const uint8_t *bit_map,
+                            bq_layout layout, void *packed, float *scales, uint8_t *zeros, void *stream) {
+  if (rows < 0 || cols < 0) return BQ_ERR_SHAPE;
+  if (wtype != BQ_F16 && wtype != BQ_BF16) return BQ_ERR_UNSUPPORTED;
+  if (layout != BQ_LAYOUT_CANONICAL && layout != BQ_LAYOUT_INTERLEAVED) return BQ_ERR_UNSUPPORTED;
+  if (rows % 128) return BQ_ERR_SHAPE;
+  if (cols % (layout == BQ_LAYOUT_CANONICAL ? 256 : 128)) return BQ_ERR_SHAPE;
+  if (rows == 0 || cols == 0) return BQ_OK;
+  if (!W || !bit_map || !packed || !scales || !zeros) return BQ_ERR_NULL;
+  if (!aligned(W, 16) || !aligned(packed, 16) || !aligned(scales, 4)) return BQ_ERR_ALIGN;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const uint16_t *w = reinterpret_cast<const uint16_t *>(W);
+  uint8_t *pk = reinterpret_cast<uint8_t *>(packed);
+  if (layout == BQ_LAYOUT_INTERLEAVED) {
+    const int64_t grid = grid_for((rows / 16) * (cols / 128));
+    if (wtype == BQ_F16) quantize_mixed_tiled_kernel<0><<<grid, kThreads, 0, st>>>(w, rows, cols, bit_map, pk, scales, zeros);
+    else quantize_mixed_tiled_kernel<1><<<grid, kThreads, 0, st>>>(w, rows, cols, bit_map, pk, scales, zeros);
+  } else {
+    const int64_t grid = grid_for(rows * (cols / 256));
+    if (wtype == BQ_F16) quantize_mixed_canonical_kernel<0><<<grid, kThreads, 0, st>>>(w, rows, cols, bit_map, pk, scales, zeros);
+    else quantize_mixed_canonical_kernel<1><<<grid, kThreads, 0, st>>>(w, rows, cols, bit_map, pk, scales, zeros);
+  }
+  return launch_status();
+}
+
+bq_status bq_dequantize(const void *packed, const float *scales, const uint8_t *zeros, const uint8_t *bit_map,
+                        int bits, int group, int64_t rows, int64_t cols, bq_layout layout, void *W_out,
+                        bq_dtype otype, void *stream) {
+  if (rows < 0 || cols < 0) return BQ_ERR_SHAPE;
+  if (otype != BQ_F16 && otype != BQ_BF16 && otype != BQ_F32) return BQ_ERR_UNSUPPORTED;
+  if (layout != BQ_LAYOUT_CANONICAL && layout != BQ_LAYOUT_INTERLEAVED) return BQ_ERR_UNSUPPORTED;
+  if (bit_map) {
+    if (rows % 128 || cols % 128) return BQ_ERR_SHAPE;
+  } else {
+    if (!valid_bits(bits)) return BQ_ERR_UNSUPPORTED;
+    if (group <= 0 || group % 8 || cols % group) return BQ_ERR_SHAPE;
+    if (layout == BQ_LAYOUT_CANONICAL) {
+      if ((cols * bits) % 32) return BQ_ERR_SHAPE;
+    } else {
+      if (group % 16 || rows % 16 || cols % tile_width(bits)) return BQ_ERR_SHAPE;
+    }
+  }
+  if (rows == 0 || cols == 0) return BQ_OK;
+  if (!packed || !scales || !zeros || !W_out) return BQ_ERR_NULL;
+  if (!aligned(packed, 16) || !aligned(W_out, 16) || !aligned(scales, 4)) return BQ_ERR_ALIGN;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const uint8_t *pk = reinterpret_cast<const uint8_t *>(packed);
+  if (bit_map) {
+    if (otype == BQ_F16) return dequant_mixed<0>(pk, scales, zeros, bit_map, rows, cols, layout, W_out, st);
+    if (otype == BQ_BF16) return dequant_mixed<1>(pk, scales, zeros, bit_map, rows, cols, layout, W_out, st);
+    return dequant_mixed<2>(pk, scales, zeros, bit_map, rows, cols, layout, W_out, st);
+  }
+  if (otype == BQ_F16) return dequant_uniform<0>(pk, scales, zeros, bits, group, rows, cols, layout, W_out, st);
+  if (otype == BQ_BF16) return dequant_uniform<1>(pk, scales, zeros, bits, group, rows, cols, layout, W_out, st);
+  return dequant_uniform<2>(pk, scales, zeros, bits, group, rows, cols, layout, W_out, st);
+}
+
+bq_status bq_linear(const void *x, bq_dtype xtype, int64_t M, int64_t K, const void *packed, const float *scales,
+                    const uint8_t *zeros, const uint8_t *bit_map, int bits, int group, int64_t N,
+                    bq_layout layout, void *y, void *stream) {
+  if (M < 0 || K < 0 || N < 0) return BQ_ERR_SHAPE;
+  if (xtype != BQ_F16 && xtype != BQ_BF16) return BQ_ERR_UNSUPPORTED;
+  if (layout != BQ_LAYOUT_INTERLEAVED) return BQ_ERR_UNSUPPORTED;
+  if (bit_map) {
+    if (N % 128 || K % 128) return BQ_ERR_SHAPE;
+  } else {
+    if (!valid_bits(bits) || !linear_group_ok(bits, group)) return BQ_ERR_UNSUPPORTED;
+    const int64_t SU = group > tile_width(bits) ? group : tile_width(bits);
+    if (N % 16 || K % SU) return BQ_ERR_SHAPE;
+  }
+  if (M == 0 || N == 0) return BQ_OK;
+  if (!x || !y) return BQ_ERR_NULL;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (K == 0) {
+    return cudaMemsetAsync(y, 0, (size_t)(M * N * 2), st) == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+  }
+  if (!packed || !scales || !zeros) return BQ_ERR_NULL;
+  if (!aligned(x, 16) || !aligned(y, 16) || !aligned(packed, 16) || !aligned(scales, 4)) return BQ_ERR_ALIGN;
+  const uint16_t *xx = reinterpret_cast<const uint16_t *>(x);
+  uint16_t *yy = reinterpret_cast<uint16_t *>(y);
+  const uint8_t *pk = reinterpret_cast<const uint8_t *>(packed);
+  // Token blocks of at most 16 go through the decode kernel.
+  for (int64_t m0 = 0; m0 < M; m0 += 16) {
+    const int mb = (int)((M - m0) < 16 ? (M - m0) : 16);
+    bq_status s = (xtype == BQ_BF16)
+                      ? gemv_dispatch<1>(xx + m0 * K, mb, K, pk, scales, zeros, bit_map, bits, group, N, yy + m0 * N, st)
+                      : gemv_dispatch<0>(xx + m0 * K, mb, K, pk, scales, zeros, bit_map, bits, group, N, yy + m0 * N, st);
+    if (s != BQ_OK) return s;
+  }
+  return BQ_OK;
+}
+
+bq_status bq_device_status(void *stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return BQ_ERR_CUDA;
+  unsigned v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_bq_status, sizeof(v)) != cudaSuccess) return BQ_ERR_CUDA;
+  if (v) {
+    const unsigned zero = 0;
+    if (cudaMemcpyToSymbol(g_bq_status, &zero, sizeof(zero)) != cudaSuccess) return BQ_ERR_CUDA;
+  }
+  if (v & BQ_FLAG_NONFINITE) return BQ_ERR_NONFINITE;
+  if (v & BQ_FLAG_BADMAP) return BQ_ERR_UNSUPPORTED;
+  if (v & BQ_FLAG_TIMEOUT) return BQ_ERR_TIMEOUT;
+  return BQ_OK;
+}
+
+}  // extern "C"

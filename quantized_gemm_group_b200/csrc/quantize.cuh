@@ -1,0 +1,338 @@
+// quantize.cuh -- group-wise asymmetric MinMax quantizer with bit packing.
+//
+// Method: GreenBitAI article ("只需单卡 RTX 3090 ..."), classic Group-wise MinMax,
+// INT4 / group 128 and INT2 / group 64; arithmetic per
+// "大模型量化实战：从原理到4-bit部署的完整指南" section 2.2 and "低比特量化",
+// section "Zero Point".  See group_params() / code_of() in common.cuh.
+//
+// HBM-bound: 2 bytes read per weight, b/8 + 5/g bytes written.  Two kernels:
+//   * canonical layout: a thread owns 8 consecutive weights (one 16-byte
+//     load), a group spans g/8 adjacent lanes and is reduced with shuffles;
+//     the thread writes its 8 codes as one 32-bit (4-bit) or 16-bit (2-bit)
+//     word.
+//   * interleaved layout: a warp owns a unit of 16 rows x U columns
+//     (U = max(tile width, g)); lane L loads exactly the weights whose codes
+//     form its own 16-byte lane slot of each 512-byte tile, so no permutation
+//     pass is needed; groups are reduced over the 4 lanes sharing a row.
+#pragma once
+#include "common.cuh"
+
+namespace bq {
+
+// ---------------------------------------------------------------------------
+// canonical layout
+// ---------------------------------------------------------------------------
+
+// Quantize 8 consecutive weights held as 4 packed 16-bit pairs; the group
+// spans LANES = G/8 adjacent lanes.  Returns the 8 codes packed LSB-first.
+template <int WT, int BITS, int G>
+BQ_DEV uint32_t quant8_canonical(uint4 v, bool active, float *s_out, uint8_t *z_out, bool *bad) {
+  using E = Elem<WT>;
+  constexpr int LANES = G / 8;
+  constexpr int QMAX = (1 << BITS) - 1;
+  uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t mn2 = E::min2(E::min2(w[0], w[1]), E::min2(w[2], w[3]));
+  uint32_t mx2 = E::max2(E::max2(w[0], w[1]), E::max2(w[2], w[3]));
+  float mn = fmin_nan(E::lo(mn2), E::hi(mn2));
+  float mx = fmax_nan(E::lo(mx2), E::hi(mx2));
+  if (!active) { mn = 0.0f; mx = 0.0f; }
+#pragma unroll
+  for (int off = 1; off < LANES; off <<= 1) {
+    mn = fmin_nan(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+    mx = fmax_nan(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  }
+  GroupParams p = group_params(mn, mx, QMAX);
+  *s_out = p.s;
+  *z_out = (uint8_t)p.z;
+  *bad = p.bad;
+  uint32_t packed = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    packed |= code_of<QMAX, WT == 0>(E::lo(w[i]), p) << (BITS * (2 * i));
+    packed |= code_of<QMAX, WT == 0>(E::hi(w[i]), p) << (BITS * (2 * i + 1));
+  }
+  return packed;
+}
+
+// W viewed flat: element e of the matrix = W[e], groups of G start at
+// multiples of G, codes packed flat.  `base_*` are the block's own arrays
+// (uniform matrix: the whole matrix).
+template <int WT, int BITS, int G, int UNROLL>
+__global__ void __launch_bounds__(256)
+quantize_canonical_kernel(const uint16_t *__restrict__ W, int64_t elems,
+                          uint8_t *__restrict__ packed, float *__restrict__ scales,
+                          uint8_t *__restrict__ zeros) {
+  constexpr int LANES = G / 8;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int64_t chunks = (elems + 255) / 256;  // 256 weights per warp step
+  bool bad_any = false;
+  for (int64_t c0 = warp * UNROLL; c0 < chunks; c0 += nwarps * UNROLL) {
+    uint4 v[UNROLL];
+    bool act[UNROLL];
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      int64_t e = (c0 + u) * 256 + lane * 8;
+      act[u] = (c0 + u < chunks) && (e < elems);
+      v[u] = act[u] ? ld_stream_v4(W + e) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      int64_t e = (c0 + u) * 256 + lane * 8;
+      float s;
+      uint8_t z;
+      bool bad;
+      uint32_t pk = quant8_canonical<WT, BITS, G>(v[u], act[u], &s, &z, &bad);
+      if (!act[u]) continue;
+      bad_any |= bad;
+      if (BITS == 4) {
+        reinterpret_cast<uint32_t *>(packed)[e / 8] = pk;
+      } else {
+        reinterpret_cast<uint16_t *>(packed)[e / 8] = (uint16_t)pk;
+      }
+      if ((lane % LANES) == 0) {
+        scales[e / G] = s;
+        zeros[e / G] = z;
+      }
+    }
+  }
+  if (bad_any) bq_flag(BQ_FLAG_NONFINITE);
+}
+
+// ---------------------------------------------------------------------------
+// interleaved (tiled) layout
+// ---------------------------------------------------------------------------
+
+template <int BITS> struct TileGeom {
+  static constexpr int T = (BITS == 4) ? 64 : 128;  // tile width in columns
+};
+
+// Field (bit offset) of the element in row half h (0: row r, 1: row r+8),
+// column pair half hp (0: columns 2c,2c+1; 1: 2c+8,2c+9), odd column `odd`,
+// 16-column run `run` inside its tile.  Returns (word index, bit offset).
+template <int BITS>
+BQ_DEV constexpr int tile_bit(int run, int h, int hp, int odd) {
+  int slot = h + 2 * hp;
+  if (BITS == 4) return 4 * (slot + 4 * odd);              // word = run
+  return 2 * (4 * (run & 1) + slot + 8 * odd);             // word = run / 2
+}
+template <int BITS>
+BQ_DEV constexpr int tile_word(int run) { return BITS == 4 ? run : run / 2; }
+
+// Process one unit: rows row0..row0+15, columns col0..col0+U-1 of a matrix
+// with K columns.  `packed` points to the matrix's packed codes, `scales` /
+// `zeros` to its [rows, K/G] metadata; all indices are relative to them.
+template <int WT, int BITS, int G>
+BQ_DEV bool quantize_unit_tiled(const uint16_t *__restrict__ W, int64_t K, int64_t row0, int64_t col0,
+                                uint8_t *__restrict__ packed, float *__restrict__ scales,
+                                uint8_t *__restrict__ zeros, int lane) {
+  using E = Elem<WT>;
+  constexpr int T = TileGeom<BITS>::T;
+  constexpr int U = (G > T) ? G : T;
+  constexpr int RUNS = U / 16;
+  constexpr int RUNS_PER_G = G / 16;
+  constexpr int NG = U / G;  // groups per row in the unit
+  constexpr int QMAX = (1 << BITS) - 1;
+  const int r = lane >> 2, c = lane & 3;
+
+  // load: [h][run][hp] half2 pairs
+  uint32_t x[2][RUNS][2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint16_t *rowp = W + (row0 + r + 8 * h) * K + col0 + 2 * c;
+#pragma unroll
+    for (int j = 0; j < RUNS; ++j) {
+      x[h][j][0] = ld_nc_u32(rowp + 16 * j);
+      x[h][j][1] = ld_nc_u32(rowp + 16 * j + 8);
+    }
+  }
+
+  bool bad_any = false;
+  GroupParams gp[2][NG];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+#pragma unroll
+    for (int gi = 0; gi < NG; ++gi) {
+      uint32_t mn2 = x[h][gi * RUNS_PER_G][0], mx2 = mn2;
+#pragma unroll
+      for (int j = gi * RUNS_PER_G; j < (gi + 1) * RUNS_PER_G; ++j) {
+#pragma unroll
+        for (int hp = 0; hp < 2; ++hp) {
+          mn2 = E::min2(mn2, x[h][j][hp]);
+          mx2 = E::max2(mx2, x[h][j][hp]);
+        }
+      }
+      float mn = fmin_nan(E::lo(mn2), E::hi(mn2));
+      float mx = fmax_nan(E::lo(mx2), E::hi(mx2));
+      mn = fmin_nan(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
+      mx = fmax_nan(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mn = fmin_nan(mn, __shfl_xor_sync(0xffffffffu, mn, 2));
+      mx = fmax_nan(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      gp[h][gi] = group_params(mn, mx, QMAX);
+      bad_any |= gp[h][gi].bad;
+    }
+  }
+
+  // codes -> lane words, tile by tile
+  constexpr int TILES = U / T;
+  constexpr int RUNS_PER_TILE = T / 16;
+#pragma unroll
+  for (int t = 0; t < TILES; ++t) {
+    uint32_t word[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int jt = 0; jt < RUNS_PER_TILE; ++jt) {
+      const int j = t * RUNS_PER_TILE + jt;
+      const int gi = j / RUNS_PER_G;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int hp = 0; hp < 2; ++hp) {
+          uint32_t pair = x[h][j][hp];
+          uint32_t q0 = code_of<QMAX, WT == 0>(E::lo(pair), gp[h][gi]);
+          uint32_t q1 = code_of<QMAX, WT == 0>(E::hi(pair), gp[h][gi]);
+          word[tile_word<BITS>(jt)] |= (q0 << tile_bit<BITS>(jt, h, hp, 0)) |
+                                       (q1 << tile_bit<BITS>(jt, h, hp, 1));
+        }
+      }
+    }
+    const int64_t tile = (row0 / 16) * (K / T) + (col0 / T) + t;
+    st_v4(packed + tile * 512 + lane * 16, make_uint4(word[0], word[1], word[2], word[3]));
+  }
+
+  if (c == 0) {
+    const int64_t GK = K / G;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+#pragma unroll
+      for (int gi = 0; gi < NG; ++gi) {
+        const int64_t idx = (row0 + r + 8 * h) * GK + col0 / G + gi;
+        scales[idx] = gp[h][gi].s;
+        zeros[idx] = (uint8_t)gp[h][gi].z;
+      }
+    }
+  }
+  return bad_any;
+}
+
+template <int WT, int BITS, int G>
+__global__ void __launch_bounds__(256)
+quantize_tiled_kernel(const uint16_t *__restrict__ W, int64_t N, int64_t K,
+                      uint8_t *__restrict__ packed, float *__restrict__ scales,
+                      uint8_t *__restrict__ zeros) {
+  constexpr int T = TileGeom<BITS>::T;
+  constexpr int U = (G > T) ? G : T;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int64_t ku = K / U;
+  const int64_t units = (N / 16) * ku;
+  bool bad = false;
+  for (int64_t u = warp; u < units; u += nwarps) {
+    const int64_t rb = u / ku, kb = u - rb * ku;
+    bad |= quantize_unit_tiled<WT, BITS, G>(W, K, rb * 16, kb * U, packed, scales, zeros, lane);
+  }
+  if (bad) bq_flag(BQ_FLAG_NONFINITE);
+}
+
+// ---------------------------------------------------------------------------
+// mixed precision: per 128-row block width from a device bit map
+// ---------------------------------------------------------------------------
+
+// Offsets of 128-row block `blk` of a mixed matrix with K columns: packed
+// byte offset and group offset, summed over the blocks before it.
+BQ_DEV void mixed_block_offsets(const uint8_t *__restrict__ bit_map, int64_t blk, int64_t K,
+                                int lane, int64_t *code_off, int64_t *group_off) {
+  int64_t sb = 0, sg = 0;
+  for (int64_t j = lane; j < blk; j += 32) {
+    int b = bit_map[j];
+    sb += b;
+    sg += (b == 4) ? 1 : 2;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    sb += __shfl_xor_sync(0xffffffffu, sb, off);
+    sg += __shfl_xor_sync(0xffffffffu, sg, off);
+  }
+  *code_off = sb * 16 * K;  // 128 rows * K cols * b / 8 bytes
+  *group_off = sg * K;      // 128 rows * K / g groups, g = 128 (b=4) or 64 (b=2)
+}
+
+template <int WT>
+__global__ void __launch_bounds__(256)
+quantize_mixed_tiled_kernel(const uint16_t *__restrict__ W, int64_t N, int64_t K,
+                            const uint8_t *__restrict__ bit_map, uint8_t *__restrict__ packed,
+                            float *__restrict__ scales, uint8_t *__restrict__ zeros) {
+  // Both production widths use 16 x 128 units: max(64, 128) and max(128, 64).
+  constexpr int U = 128;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int64_t ku = K / U;
+  const int64_t units = (N / 16) * ku;
+  bool bad = false, badmap = false;
+  for (int64_t u = warp; u < units; u += nwarps) {
+    const int64_t rb = u / ku, kb = u - rb * ku;
+    const int64_t blk = rb / 8;
+    const int bits = bit_map[blk];
+    int64_t co, go;
+    mixed_block_offsets(bit_map, blk, K, lane, &co, &go);
+    const int64_t row_in_blk = (rb % 8) * 16;
+    const uint16_t *Wb = W + blk * 128 * K;
+    if (bits == 4) {
+      bad |= quantize_unit_tiled<WT, 4, 128>(Wb, K, row_in_blk, kb * U, packed + co, scales + go,
+                                             zeros + go, lane);
+    } else if (bits == 2) {
+      bad |= quantize_unit_tiled<WT, 2, 64>(Wb, K, row_in_blk, kb * U, packed + co, scales + go,
+                                            zeros + go, lane);
+    } else {
+      badmap = true;
+    }
+  }
+  if (bad) bq_flag(BQ_FLAG_NONFINITE);
+  if (badmap) bq_flag(BQ_FLAG_BADMAP);
+}
+
+// Canonical mixed: a warp quantizes 256 consecutive weights of one row; the
+// block's codes are flat within its own 128 x K region.
+template <int WT>
+__global__ void __launch_bounds__(256)
+quantize_mixed_canonical_kernel(const uint16_t *__restrict__ W, int64_t N, int64_t K,
+                                const uint8_t *__restrict__ bit_map, uint8_t *__restrict__ packed,
+                                float *__restrict__ scales, uint8_t *__restrict__ zeros) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int64_t per_row = K / 256;
+  const int64_t chunks = N * per_row;
+  bool bad_any = false, badmap = false;
+  for (int64_t ch = warp; ch < chunks; ch += nwarps) {
+    const int64_t row = ch / per_row, kc = ch - row * per_row;
+    const int64_t blk = row / 128;
+    const int bits = bit_map[blk];
+    int64_t co, go;
+    mixed_block_offsets(bit_map, blk, K, lane, &co, &go);
+    const int64_t e_in_blk = (row % 128) * K + kc * 256 + lane * 8;  // flat index inside block
+    uint4 v = ld_stream_v4(W + blk * 128 * K + e_in_blk);
+    float s;
+    uint8_t z;
+    bool bad;
+    if (bits == 4) {
+      uint32_t pk = quant8_canonical<WT, 4, 128>(v, true, &s, &z, &bad);
+      reinterpret_cast<uint32_t *>(packed + co)[e_in_blk / 8] = pk;
+      if ((lane % 16) == 0) { scales[go + e_in_blk / 128] = s; zeros[go + e_in_blk / 128] = z; }
+      bad_any |= bad;
+    } else if (bits == 2) {
+      uint32_t pk = quant8_canonical<WT, 2, 64>(v, true, &s, &z, &bad);
+      reinterpret_cast<uint16_t *>(packed + co)[e_in_blk / 8] = (uint16_t)pk;
+      if ((lane % 8) == 0) { scales[go + e_in_blk / 64] = s; zeros[go + e_in_blk / 64] = z; }
+      bad_any |= bad;
+    } else {
+      badmap = true;
+    }
+  }
+  if (bad_any) bq_flag(BQ_FLAG_NONFINITE);
+  if (badmap) bq_flag(BQ_FLAG_BADMAP);
+}
+
+}  // namespace bq
