@@ -359,6 +359,8 @@ def run_gpu(args, world, rank, local):
     dist_kind = "t4" if args.bits == 2 else "normal"
     stack = Stack(args.layers, bits, group, seed_offset=rank * 100000, dist_kind=dist_kind,
                   quant_time=not args.no_quant)
+    torch.cuda.synchronize()
+    bq.bq_set_option(bq.BQ_OPT_LINEAR_OVERLAP, args.overlap)
     Ms = M_SET
     xs = {M: [synth.activations(M, K, seed=10000 * M + i + rank * 7, device="cuda")
               for i, (_, _, _, N, K) in enumerate(stack.shapes)] for M in Ms}
@@ -420,7 +422,8 @@ def run_gpu(args, world, rank, local):
                    "weights": "fp16 N(0,0.02)" if bits == 4 else "fp16 Student-t4 std 0.02 + 0.1% x10 outlier cols",
                    "activations": "bf16 N(0,1)", "l2": "inputs larger than L2 (packed stack %.2f GB)" %
                    (sum(weight_bytes(N, K, bits, group) for (_, _, _, N, K) in stack.shapes) / 1e9),
-                   "graph": "one CUDA graph per step", "parallelism": f"replicas x{world} (independent batches)"},
+                   "graph": "one CUDA graph per step", "overlap": args.overlap,
+                   "parallelism": f"replicas x{world} (independent batches)"},
         "roofline": roofline,
         "clocks": clocks,
         "e2e": {"value": round(world * step_bytes / t_e2e / 1e9, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
@@ -501,6 +504,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-quant", action="store_true")
     ap.add_argument("--quick", action="store_true", help="skip the per-shape breakdown")
+    ap.add_argument("--overlap", type=int, default=2, choices=[0, 1, 2],
+                    help="bq_linear launch overlap: 0 plain, 1 programmatic dependent launch, "
+                         "2 PDL + weight streaming before the wait (weights are static here)")
     args = ap.parse_args()
 
     world, rank, local = dist_setup()

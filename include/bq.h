@@ -72,7 +72,12 @@ typedef enum { BQ_F16 = 0, BQ_BF16 = 1, BQ_F32 = 2 } bq_dtype;
  *
  * BQ_LAYOUT_INTERLEAVED: the layout the linear kernels read.  The matrix is
  *   cut into 512-byte tiles of 16 rows by T columns (T = 64 for 4-bit, 128 for
- *   2-bit), stored row-block major (tile (rb, kt) at 512 * (rb * cols/T + kt)).
+ *   2-bit).  Rows are grouped in blocks of 128 (the last block may be shorter:
+ *   R_b = its rows / 16 tiles high).  Block b starts at byte
+ *   b * 128 * cols * bits / 8 and stores its tiles column-block major: tile
+ *   (row tile t of the block, column block kt) at 512 * (kt * R_b + t) from
+ *   the block start, so a run of column blocks of a whole block is one
+ *   contiguous range.
  *   Inside a tile, 16-byte "lane" L (0..31) serves rows r = L/4 and r + 8 and,
  *   in every run of 16 columns, the column pairs (2c, 2c+1) and (2c+8, 2c+9),
  *   c = L % 4.  Slot i of a run is (row r, low pair), (row r+8, low pair),
@@ -82,6 +87,11 @@ typedef enum { BQ_F16 = 0, BQ_BF16 = 1, BQ_F32 = 2 } bq_dtype;
  *     2-bit: word j holds runs 2j (fields 0..3, 8..11) and 2j+1 (fields
  *            4..7, 12..15); slot i of run 2j+h keeps its even column in field
  *            4h + i and its odd column in field 4h + i + 8.
+ *   Scales and zeros of the interleaved layout are stored 128-row-block
+ *   major, then by group, then by row: group g of row n (G = cols / group
+ *   groups per row) at index 128 * G * (n / 128) + g * R + n % 128, R = rows
+ *   of n's block, so a block's metadata over a run of groups is contiguous.
+ *   (Canonical layout: row-major [rows, cols/group].)
  *   Needs rows % 16 == 0 and cols % T == 0.  With this order a lane's 16-byte
  *   load is already in the register order of a 16x8x16 bf16 tensor-core
  *   fragment, and one AND/OR with a magic exponent turns two codes into a
@@ -120,8 +130,8 @@ bq_status bq_mixed_offsets(const uint8_t *bit_map, int64_t rows, int64_t cols,
  *            also 8).
  *   layout   BQ_LAYOUT_CANONICAL or BQ_LAYOUT_INTERLEAVED (shape rules above)
  *   packed   [bq_packed_bytes(rows, cols, bits)] bytes, 16-byte aligned
- *   scales   [rows, cols/group] fp32
- *   zeros    [rows, cols/group] uint8
+ *   scales   rows * cols/group fp32, in the layout's metadata order (above)
+ *   zeros    rows * cols/group uint8, same order
  * A non-finite weight, or a group whose scale overflows fp32, sets
  * BQ_ERR_NONFINITE in the device status word; that group's outputs are then
  * unspecified.
@@ -156,7 +166,8 @@ bq_status bq_dequantize(const void *packed, const float *scales, const uint8_t *
 /*
  * bq_linear: y[M, N] = x[M, K] . dequant(W)^T.
  *   x        [M, K] of xtype (BQ_BF16 or BQ_F16), 16-byte aligned rows (K % 8 == 0)
- *   packed / scales / zeros: from bq_quantize in BQ_LAYOUT_INTERLEAVED
+ *   packed / scales / zeros: from bq_quantize in BQ_LAYOUT_INTERLEAVED; all
+ *            three 16-byte aligned (they are read with bulk copies)
  *   bit_map  NULL for a uniform matrix (bits, group used; production pairs
  *            (4, 128) and (2, 64), tests also group 32 and 256), else a DEVICE
  *            bit map as in bq_quantize_mixed (bits, group ignored)
@@ -164,8 +175,9 @@ bq_status bq_dequantize(const void *packed, const float *scales, const uint8_t *
  * Products are accumulated in fp32 per group on exact (q - z) operands, then
  * scaled by the group's fp32 s and summed in fp32; y is rounded once.
  * M <= 16 runs the decode kernel (split-K dequant-GEMV on tensor cores);
- * larger M runs the prefill kernel.  Needs N % 16 == 0 (N % 128 == 0 with a
- * bit map) and K a multiple of the tile width of every width used.
+ * larger M runs the prefill kernel.  Needs N % 16 == 0 and K % 256 == 0 at
+ * 4 bits, K % 512 == 0 at 2 bits; with a bit map N % 128 == 0 and
+ * K % 512 == 0.
  */
 bq_status bq_linear(const void *x, bq_dtype xtype, int64_t M, int64_t K,
                     const void *packed, const float *scales, const uint8_t *zeros,
@@ -173,10 +185,46 @@ bq_status bq_linear(const void *x, bq_dtype xtype, int64_t M, int64_t K,
                     bq_layout layout, void *y, void *stream);
 
 /*
+ * Options.
+ *
+ * BQ_OPT_LINEAR_OVERLAP (process-wide, default 0 or the value of the
+ * environment variable BQ_OVERLAP):
+ *   0  bq_linear launches plainly.
+ *   1  bq_linear uses programmatic dependent launch: it lets the next kernel
+ *      in the stream start launching early and waits for the previous kernel
+ *      to complete before reading any input or writing y.  Hides launch gaps
+ *      in back-to-back layers; results are identical.
+ *   2  as 1, and the decode kernel may start streaming packed codes, scales
+ *      and zeros BEFORE the previous kernel in the stream has completed.  Only
+ *      valid when that kernel does not write them (static weights, e.g. a
+ *      decode step); x is always read after the wait.
+ * bq_set_option returns BQ_ERR_UNSUPPORTED for an unknown option or value.
+ */
+typedef enum { BQ_OPT_LINEAR_OVERLAP = 0 } bq_option;
+bq_status bq_set_option(int option, int value);
+int bq_get_option(int option);
+
+/*
  * bq_device_status: synchronize `stream`, return the first error recorded by
  * a kernel since the last call (BQ_OK if none) and clear it.
  */
 bq_status bq_device_status(void *stream);
+
+/*
+ * bq_check_division: diagnostic.  The quantizer rounds x / s from a quotient
+ * computed by two Markstein refinements of x * RN(1/s) (P. Markstein, IBM J.
+ * Res. Dev. 34(1), 1990) rather than an IEEE division.  This entry point
+ * compares that quotient (with `refinements` = 1 or 2 steps) bit for bit
+ * against the IEEE division (a zero quotient of either sign counts as equal:
+ * x = -0 gives +0 after refinement, and both round to the same code) for
+ * every fp32 divisor whose bit pattern lies in
+ * [s_bits_begin, s_bits_end) and every fp16 numerator with |x| < 64.
+ *   result  DEVICE array of 4 uint64, zeroed by the caller: [0] mismatches,
+ *           [1] pairs checked, [2] / [3] bit patterns of the first mismatch
+ *           found (divisor, fp16 numerator).
+ */
+bq_status bq_check_division(uint32_t s_bits_begin, uint32_t s_bits_end, int refinements,
+                            unsigned long long *result, void *stream);
 
 /* Human-readable name of a status code (static string). */
 const char *bq_status_string(bq_status status);

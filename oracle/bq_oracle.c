@@ -188,11 +188,14 @@ static void canonical_position(int64_t n, int64_t k, int64_t cols, int bits,
 /* Interleaved (tiled) layout used by the linear kernels.
  *
  * The matrix is cut into tiles of 16 rows by T columns (T = 64 for 4-bit,
- * T = 128 for 2-bit); every tile is 512 bytes.  Tiles are stored row-block
- * major: tile (row block rb, column block kt) starts at byte
- * 512 * (rb * (cols/T) + kt).  Inside a tile, "lane" L in 0..31 owns bytes
- * [16L, 16L + 16) = four 32-bit words.  Lane L serves rows r = L/4 and r + 8 of
- * the tile and, within each run of 16 columns, the column pairs (2c, 2c+1)
+ * T = 128 for 2-bit); every tile is 512 bytes.  Rows are grouped in blocks
+ * of 128 (8 tiles high; the last block may hold fewer, R_b = its rows / 16).
+ * Block b starts at byte b * 128 * cols * bits / 8 and stores its tiles
+ * column-block major: tile (row tile t of the block, column block kt) at
+ * 512 * (kt * R_b + t) from the block start, so one column block of a whole
+ * 128-row block is contiguous.  Inside a tile, "lane" L in 0..31 owns bytes
+ * [16L, 16L + 16) = four 32-bit words.  Lane L serves rows r = L/4 and r + 8
+ * of the tile and, within each run of 16 columns, the column pairs (2c, 2c+1)
  * and (2c+8, 2c+9) with c = L % 4.  The four (row, column pair) slots of one
  * run of 16 columns are numbered
  *     slot 0: row r,   columns 2c, 2c+1
@@ -206,11 +209,21 @@ static void canonical_position(int64_t n, int64_t k, int64_t cols, int bits,
  *        field 4h + i + 8.
  * Fields are numbered from the least significant bit of the little-endian
  * 32-bit word. */
-static void interleaved_position(int64_t n, int64_t k, int64_t cols, int bits,
+static int64_t block_rows(int64_t n, int64_t rows)
+{
+    int64_t b = n / 128;
+    int64_t left = rows - b * 128;
+    return left < 128 ? left : 128;
+}
+
+static void interleaved_position(int64_t n, int64_t k, int64_t rows, int64_t cols, int bits,
                                  int64_t *byte_off, int *bit_off)
 {
     const int64_t T = (bits == 4) ? 64 : 128;
-    int64_t rb = n / 16, kt = k / T;
+    int64_t b = n / 128;
+    int64_t Rb = block_rows(n, rows) / 16;   /* row tiles in this block */
+    int64_t t = (n % 128) / 16;              /* row tile inside the block */
+    int64_t kt = k / T;
     int rr = (int)(n % 16);
     int kk = (int)(k % T);
     int r = rr % 8, upper_row = rr / 8;
@@ -230,24 +243,24 @@ static void interleaved_position(int64_t n, int64_t k, int64_t cols, int bits,
         field = 4 * (run % 2) + slot + 8 * odd;
     }
     int bit_in_word = field * bits;
-    int64_t tile = rb * (cols / T) + kt;
-    *byte_off = tile * 512 + lane * 16 + word * 4 + bit_in_word / 8;
+    int64_t block_start = b * 128 * cols * bits / 8;
+    *byte_off = block_start + (kt * Rb + t) * 512 + lane * 16 + word * 4 + bit_in_word / 8;
     *bit_off = bit_in_word % 8;
 }
 
-static void position(int layout, int64_t n, int64_t k, int64_t cols, int bits,
+static void position(int layout, int64_t n, int64_t k, int64_t rows, int64_t cols, int bits,
                      int64_t *byte_off, int *bit_off)
 {
     if (layout == 0) canonical_position(n, k, cols, bits, byte_off, bit_off);
-    else interleaved_position(n, k, cols, bits, byte_off, bit_off);
+    else interleaved_position(n, k, rows, cols, bits, byte_off, bit_off);
 }
 
-/* Byte offset and bit offset of element (n, k): exported so tests can check
- * the map against hand-derived positions. */
-void bqo_code_position(int layout, int64_t n, int64_t k, int64_t cols, int bits,
+/* Byte offset and bit offset of element (n, k) of a rows x cols matrix:
+ * exported so tests can check the map against hand-derived positions. */
+void bqo_code_position(int layout, int64_t n, int64_t k, int64_t rows, int64_t cols, int bits,
                        int64_t *byte_off, int *bit_off)
 {
-    position(layout, n, k, cols, bits, byte_off, bit_off);
+    position(layout, n, k, rows, cols, bits, byte_off, bit_off);
 }
 
 int bqo_pack(const uint8_t *codes, int64_t rows, int64_t cols, int bits,
@@ -266,7 +279,7 @@ int bqo_pack(const uint8_t *codes, int64_t rows, int64_t cols, int bits,
         for (int64_t k = 0; k < cols; ++k) {
             int64_t byte_off;
             int bit_off;
-            position(layout, n, k, cols, bits, &byte_off, &bit_off);
+            position(layout, n, k, rows, cols, bits, &byte_off, &bit_off);
             out[byte_off] |= (uint8_t)((codes[n * cols + k] & mask) << bit_off);
         }
     }
@@ -282,11 +295,35 @@ int bqo_unpack(const uint8_t *packed, int64_t rows, int64_t cols, int bits,
         for (int64_t k = 0; k < cols; ++k) {
             int64_t byte_off;
             int bit_off;
-            position(layout, n, k, cols, bits, &byte_off, &bit_off);
+            position(layout, n, k, rows, cols, bits, &byte_off, &bit_off);
             codes[n * cols + k] = (uint8_t)((packed[byte_off] >> bit_off) & mask);
         }
     }
     return BQO_OK;
+}
+
+/* Metadata layout.  Canonical: scales / zeros are [rows, cols/group],
+ * row-major.  Interleaved: 128-row-block major, then group, then row, so the
+ * metadata of one 128-row block over a run of groups is contiguous: element
+ * (n, g) of a matrix with G groups per row sits at index
+ * 128 * G * (n / 128) + g * R + n % 128, where R is the number of rows of
+ * n's block (128, or fewer in a last partial block). */
+int64_t bqo_meta_index(int layout, int64_t n, int64_t g, int64_t rows, int64_t G)
+{
+    if (layout == 0) return n * G + g;
+    return 128 * G * (n / 128) + g * block_rows(n, rows) + n % 128;
+}
+
+void bqo_pack_meta_f32(const float *in, int64_t rows, int64_t G, int layout, float *out)
+{
+    for (int64_t n = 0; n < rows; ++n)
+        for (int64_t g = 0; g < G; ++g) out[bqo_meta_index(layout, n, g, rows, G)] = in[n * G + g];
+}
+
+void bqo_pack_meta_u8(const uint8_t *in, int64_t rows, int64_t G, int layout, uint8_t *out)
+{
+    for (int64_t n = 0; n < rows; ++n)
+        for (int64_t g = 0; g < G; ++g) out[bqo_meta_index(layout, n, g, rows, G)] = in[n * G + g];
 }
 
 /* ------------------------------------------------------------------ */

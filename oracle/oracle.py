@@ -54,7 +54,7 @@ def lib():
             L.bqo_quantize_group.restype = i32
             L.bqo_quantize.argtypes = [vp, i32, i64, i64, i32, i32, i64, i64, vp, vp, vp]
             L.bqo_quantize.restype = i32
-            L.bqo_code_position.argtypes = [i32, i64, i64, i64, i32, vp, vp]
+            L.bqo_code_position.argtypes = [i32, i64, i64, i64, i64, i32, vp, vp]
             L.bqo_code_position.restype = None
             L.bqo_pack.argtypes = [vp, i64, i64, i32, i32, vp]
             L.bqo_pack.restype = i32
@@ -68,6 +68,12 @@ def lib():
             L.bqo_linear_f64.restype = None
             L.bqo_decode_f64.argtypes = [vp, i32, i64, vp]
             L.bqo_decode_f64.restype = None
+            L.bqo_meta_index.argtypes = [i32, i64, i64, i64, i64]
+            L.bqo_meta_index.restype = i64
+            L.bqo_pack_meta_f32.argtypes = [vp, i64, i64, i32, vp]
+            L.bqo_pack_meta_f32.restype = None
+            L.bqo_pack_meta_u8.argtypes = [vp, i64, i64, i32, vp]
+            L.bqo_pack_meta_u8.restype = None
             L.bqo_f64_to_bf16.argtypes = [ctypes.c_double]
             L.bqo_f64_to_bf16.restype = ctypes.c_uint16
             _lib = L
@@ -171,10 +177,10 @@ def quantize(w_bits: np.ndarray, wtype: str, bits: int, group: int, threads: int
 # packing
 # ---------------------------------------------------------------------------
 
-def code_position(layout: str, n: int, k: int, cols: int, bits: int):
+def code_position(layout: str, n: int, k: int, rows: int, cols: int, bits: int):
     b = ctypes.c_int64()
     o = ctypes.c_int()
-    lib().bqo_code_position(LAYOUT[layout], n, k, cols, bits, ctypes.byref(b), ctypes.byref(o))
+    lib().bqo_code_position(LAYOUT[layout], n, k, rows, cols, bits, ctypes.byref(b), ctypes.byref(o))
     return int(b.value), int(o.value)
 
 
@@ -195,6 +201,22 @@ def unpack(packed: np.ndarray, N: int, K: int, bits: int, layout: str) -> np.nda
     if rc:
         raise OracleError(f"bqo_unpack rc={rc}")
     return codes
+
+
+def meta_index(layout: str, n: int, g: int, rows: int, G: int) -> int:
+    return int(lib().bqo_meta_index(LAYOUT[layout], n, g, rows, G))
+
+
+def pack_meta(scales: np.ndarray, zeros: np.ndarray, layout: str):
+    """Scales / zeros [rows, G] -> the layout's flat storage order."""
+    scales = np.ascontiguousarray(scales, dtype=np.float32)
+    zeros = np.ascontiguousarray(zeros, dtype=np.uint8)
+    rows, G = scales.shape
+    s = np.empty(rows * G, dtype=np.float32)
+    z = np.empty(rows * G, dtype=np.uint8)
+    lib().bqo_pack_meta_f32(_p(scales), rows, G, LAYOUT[layout], _p(s))
+    lib().bqo_pack_meta_u8(_p(zeros), rows, G, LAYOUT[layout], _p(z))
+    return s, z
 
 
 # ---------------------------------------------------------------------------
@@ -284,8 +306,9 @@ def quantize_mixed(w_bits: np.ndarray, wtype: str, bit_map, layout: str, threads
         blk = w_bits[i * MIX_BLOCK:(i + 1) * MIX_BLOCK]
         c, s, z = quantize(blk, wtype, b, GROUP_OF_BITS[b], threads)
         packed.append(pack(c, b, layout))
-        scales.append(s.reshape(-1))
-        zeros.append(z.reshape(-1))
+        ms, mz = pack_meta(s, z, layout)
+        scales.append(ms)
+        zeros.append(mz)
         codes_blocks.append((c, s, z))
     return (np.concatenate(packed), np.concatenate(scales), np.concatenate(zeros), codes_blocks)
 

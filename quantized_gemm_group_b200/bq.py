@@ -32,8 +32,10 @@ GROUP_OF_BITS = {4: 128, 2: 64}
 #: every symbol include/bq.h declares
 EXPORTS = (
     "bq_packed_bytes", "bq_group_count", "bq_mixed_offsets", "bq_quantize", "bq_quantize_mixed",
-    "bq_dequantize", "bq_linear", "bq_device_status", "bq_status_string", "bq_version",
+    "bq_dequantize", "bq_linear", "bq_check_division", "bq_set_option", "bq_get_option", "bq_device_status",
+    "bq_status_string", "bq_version",
 )
+BQ_OPT_LINEAR_OVERLAP = 0
 
 
 class BQError(RuntimeError):
@@ -70,6 +72,12 @@ def lib(path: str | None = None):
     L.bq_dequantize.restype = i32
     L.bq_linear.argtypes = [vp, i32, i64, i64, vp, vp, vp, vp, i32, i32, i64, i32, vp, vp]
     L.bq_linear.restype = i32
+    L.bq_check_division.argtypes = [ctypes.c_uint32, ctypes.c_uint32, i32, vp, vp]
+    L.bq_check_division.restype = i32
+    L.bq_set_option.argtypes = [i32, i32]
+    L.bq_set_option.restype = i32
+    L.bq_get_option.argtypes = [i32]
+    L.bq_get_option.restype = i32
     L.bq_device_status.argtypes = [vp]
     L.bq_device_status.restype = i32
     L.bq_status_string.argtypes = [i32]
@@ -128,13 +136,15 @@ def bq_mixed_offsets(bit_map, rows: int, cols: int):
 
 def bq_quantize(W: torch.Tensor, bits: int, group: int | None = None, layout: str = "interleaved",
                 out=None, stream=None):
-    """Quantize W [N, K] (fp16/bf16, CUDA).  Returns (packed u8, scales f32 [N, K/g], zeros u8 [N, K/g])."""
+    """Quantize W [N, K] (fp16/bf16, CUDA).  Returns (packed u8, scales f32, zeros u8): scales / zeros
+    are [N, K/g] in the canonical layout and flat (16-row-block-major order) in the interleaved one."""
     group = group or GROUP_OF_BITS[bits]
     N, K = W.shape
     if out is None:
         packed = torch.empty(max(1, bq_packed_bytes(N, K, bits)), dtype=torch.uint8, device=W.device)
-        scales = torch.empty((N, K // group), dtype=torch.float32, device=W.device)
-        zeros = torch.empty((N, K // group), dtype=torch.uint8, device=W.device)
+        mshape = (N, K // group) if layout == "canonical" else (N * (K // group),)
+        scales = torch.empty(mshape, dtype=torch.float32, device=W.device)
+        zeros = torch.empty(mshape, dtype=torch.uint8, device=W.device)
     else:
         packed, scales, zeros = out
     st = lib().bq_quantize(_ptr(W), DTYPE_CODE[W.dtype], N, K, bits, group, LAYOUTS[layout],
@@ -183,6 +193,23 @@ def bq_linear(x: torch.Tensor, packed, scales, zeros, N: int, bits: int = 4, gro
                          _ptr(bit_map_dev), bits, group, N, LAYOUTS[layout], _ptr(y), _stream(stream))
     _check("bq_linear", st)
     return y
+
+
+def bq_check_division(s_bits_begin: int, s_bits_end: int, refinements: int = 2, stream=None):
+    """Returns (mismatches, pairs checked, first bad divisor bits, first bad fp16 numerator bits)."""
+    res = torch.zeros(4, dtype=torch.int64, device="cuda")
+    _check("bq_check_division", lib().bq_check_division(s_bits_begin, s_bits_end, refinements, _ptr(res),
+                                                        _stream(stream)))
+    torch.cuda.synchronize()
+    return tuple(int(v) for v in res.cpu())
+
+
+def bq_set_option(option: int, value: int):
+    _check("bq_set_option", lib().bq_set_option(option, value))
+
+
+def bq_get_option(option: int) -> int:
+    return int(lib().bq_get_option(option))
 
 
 def bq_device_status(stream=None) -> int:

@@ -11,6 +11,7 @@
 #include "dequant.cuh"
 #include "gemv.cuh"
 #include "quantize.cuh"
+#include "selftest.cuh"
 
 using namespace bq;
 
@@ -128,88 +129,117 @@ bq_status dequant_mixed(const uint8_t *packed, const float *scales, const uint8_
 // GEMV (M <= 16) geometry and dispatch
 // ---------------------------------------------------------------------------
 
-struct Geom {
-  int NB, R, NWR, NWK, S;
-  int64_t KC, KW;
-};
+// 0: plain launches; 1: programmatic dependent launch (the kernel waits for
+// the previous one before reading anything); 2: as 1, and weights may be
+// streamed before that wait (the caller guarantees the preceding kernel does
+// not write them).
+int g_overlap_mode = -1;
 
-bool pdl_enabled() {
-  static int v = -1;
-  if (v < 0) {
-    const char *e = getenv("BQ_PDL");
-    v = (e && e[0] == '1') ? 1 : 0;
+int overlap_mode() {
+  if (g_overlap_mode < 0) {
+    const char *e = getenv("BQ_OVERLAP");
+    g_overlap_mode = (e && (e[0] == '1' || e[0] == '2')) ? e[0] - '0' : 0;
   }
-  return v == 1;
+  return g_overlap_mode;
 }
 
-Geom gemv_geometry(int M, int64_t N, int64_t K, int64_t SU, bool mixed) {
-  Geom g;
+struct GemvGeom {
+  int NB, SK, stages;
+  int64_t KC;
+};
+
+constexpr int kTwoCtaSmem = 112 * 1024;   // per-CTA budget that keeps two CTAs per SM
+constexpr int kMaxSmem = 227 * 1024;
+
+int deepest_ring(int M, int tok, int64_t kc, int groups, int budget) {
+  for (int cand = kGemvMaxStages; cand >= 2; --cand)
+    if (gemv_smem_layout(M, tok, kc, groups, cand).total <= budget) return cand;
+  return 0;
+}
+
+// Split-K S_k (CTAs per cluster, dividing K / SC, at most 8) and ring depth.
+// Preferred: the smallest split that gives every SM a CTA while two CTAs
+// still fit per SM.  Otherwise the largest split that fits two CTAs per SM
+// (more CTAs, more bytes in flight); otherwise the largest that fits at all.
+// G_max: the smallest group size the kernel may meet (most metadata).
+GemvGeom gemv_geometry(int M, int64_t N, int64_t K, int SC, int G_min) {
+  GemvGeom g;
   g.NB = (M <= 8) ? 1 : 2;
-  g.R = (N % 32 == 0) ? 2 : 1;
-  g.NWR = 1;
-  for (int c : {4, 2, 1}) {
-    if (N % (16 * g.R * c) == 0) { g.NWR = c; break; }
-  }
-  if (mixed) { g.R = 2; g.NWR = 4; }
-  const int64_t rows = 16 * g.R * g.NWR;
-  const int64_t row_ctas = N / rows;
-  const int64_t units = K / SU;
-  const int64_t target_warps = (int64_t)sm_count() * 14;
-  const int max_nwk = 8 / g.NWR;
-  // smallest split d = S * NWK (S <= 8 CTAs per cluster, NWK <= max_nwk
-  // warps along K) dividing the units that reaches the target warp count
-  int best_s = 1, best_nwk = 1;
-  for (int d = 1; d <= 8 * max_nwk; ++d) {
-    if (units % d) continue;
-    int nwk = 0;
-    for (int c = 1; c <= max_nwk; ++c) {
-      if (d % c == 0 && d / c <= 8) { nwk = c; break; }
+  const int tok = 8 * g.NB;
+  const int64_t rc = (N + 127) / 128;
+  const int64_t nst = K / SC;
+  const int64_t sms = sm_count();
+  int best2 = -1, best2_st = 0, best1 = -1, best1_st = 0;
+  for (int d = 1; d <= 8; ++d) {
+    if (nst % d) continue;
+    const int64_t kc = K / d;
+    const int groups = (int)(kc / G_min);
+    const int st2 = deepest_ring(M, tok, kc, groups, kTwoCtaSmem);
+    if (st2) {
+      if (rc * d >= sms) {
+        g.SK = d;
+        g.stages = st2;
+        g.KC = kc;
+        return g;
+      }
+      best2 = d;
+      best2_st = st2;
     }
-    if (!nwk) continue;
-    best_s = d / nwk;
-    best_nwk = nwk;
-    if (row_ctas * g.NWR * d >= target_warps) break;
+    const int st1 = deepest_ring(M, tok, kc, groups, kMaxSmem);
+    if (st1) {
+      best1 = d;
+      best1_st = st1;
+    }
   }
-  g.NWK = best_nwk;
-  g.S = best_s;
-  g.KC = K / g.S;
-  g.KW = g.KC / g.NWK;
+  if (best2 > 0) {
+    g.SK = best2;
+    g.stages = best2_st;
+  } else if (best1 > 0) {
+    g.SK = best1;
+    g.stages = best1_st;
+  } else {
+    g.SK = 8;
+    g.stages = 2;
+  }
+  g.KC = K / g.SK;
   return g;
 }
 
-template <int XT, int BITS, int G, int NB, int R, bool MIXED>
-bq_status launch_gemv_t(const Geom &g, const uint16_t *x, int M, int64_t K, const uint8_t *packed,
-                        const float *scales, const uint8_t *zeros, const uint8_t *bit_map, int64_t N,
-                        uint16_t *y, cudaStream_t st) {
-  auto kern = gemv_kernel<XT, BITS, G, NB, R, MIXED>;
-  const size_t smem = gemv_smem_bytes(NB, R, g.NWR, g.NWK, g.KC);
+template <int XT, int BITS, int G, int NB, bool MIXED>
+bq_status launch_gemv_t(const GemvGeom &g, GemvArgs a, int G_min, cudaStream_t st) {
+  auto kern = gemv_kernel<XT, BITS, G, NB, MIXED>;
   static bool attr_set = false;
   if (!attr_set) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem) != cudaSuccess)
       return BQ_ERR_CUDA;
     attr_set = true;
   }
-  if (smem > 227 * 1024) return BQ_ERR_SHAPE;
+  a.stages = g.stages;
+  a.KC = g.KC;
+  a.L = gemv_smem_layout(a.M, 8 * NB, g.KC, (int)(g.KC / G_min), g.stages);
+  if (a.L.total > kMaxSmem) return BQ_ERR_SHAPE;
+  const int mode = overlap_mode();
+  a.prefetch_before_wait = (mode == 2) ? 1 : 0;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(N / (16 * R * g.NWR)), (unsigned)g.S, 1);
-  cfg.blockDim = dim3((unsigned)(32 * g.NWR * g.NWK), 1, 1);
-  cfg.dynamicSmemBytes = smem;
+  cfg.gridDim = dim3((unsigned)((a.N + 127) / 128), (unsigned)g.SK, 1);
+  cfg.blockDim = dim3(32 * (kGemvMaxConsumers + 1), 1, 1);
+  cfg.dynamicSmemBytes = (size_t)a.L.total;
   cfg.stream = st;
   cudaLaunchAttribute attrs[2];
   int na = 0;
   attrs[na].id = cudaLaunchAttributeClusterDimension;
   attrs[na].val.clusterDim.x = 1;
-  attrs[na].val.clusterDim.y = (unsigned)g.S;
+  attrs[na].val.clusterDim.y = (unsigned)g.SK;
   attrs[na].val.clusterDim.z = 1;
   ++na;
-  if (pdl_enabled()) {
+  if (mode >= 1) {
     attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attrs[na].val.programmaticStreamSerializationAllowed = 1;
     ++na;
   }
   cfg.attrs = attrs;
   cfg.numAttrs = na;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, x, M, K, packed, scales, zeros, bit_map, N, y, g.KC, g.KW, g.NWR);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return BQ_ERR_CUDA;
@@ -217,31 +247,35 @@ bq_status launch_gemv_t(const Geom &g, const uint16_t *x, int M, int64_t K, cons
   return BQ_OK;
 }
 
+// Stage width: 256 columns at 4 bits, 512 at 2 bits; a mixed matrix uses
+// 512-column splits so that both widths tile every CTA's slice.
 template <int XT, int BITS, int G, bool MIXED>
-bq_status launch_gemv_nb(const Geom &g, const uint16_t *x, int M, int64_t K, const uint8_t *packed,
-                         const float *scales, const uint8_t *zeros, const uint8_t *bit_map, int64_t N,
-                         uint16_t *y, cudaStream_t st) {
-  if (g.NB == 1) {
-    if (g.R == 2) return launch_gemv_t<XT, BITS, G, 1, 2, MIXED>(g, x, M, K, packed, scales, zeros, bit_map, N, y, st);
-    return launch_gemv_t<XT, BITS, G, 1, 1, MIXED>(g, x, M, K, packed, scales, zeros, bit_map, N, y, st);
-  }
-  if (g.R == 2) return launch_gemv_t<XT, BITS, G, 2, 2, MIXED>(g, x, M, K, packed, scales, zeros, bit_map, N, y, st);
-  return launch_gemv_t<XT, BITS, G, 2, 1, MIXED>(g, x, M, K, packed, scales, zeros, bit_map, N, y, st);
+bq_status launch_gemv_dispatch(const GemvArgs &a, cudaStream_t st) {
+  const int split_unit = MIXED ? 512 : StageG<BITS, G>::SC;
+  if (a.K % split_unit) return BQ_ERR_SHAPE;
+  const int G_min = MIXED ? 64 : G;
+  GemvGeom g = gemv_geometry(a.M, a.N, a.K, split_unit, G_min);
+  if (g.NB == 1) return launch_gemv_t<XT, BITS, G, 1, MIXED>(g, a, G_min, st);
+  return launch_gemv_t<XT, BITS, G, 2, MIXED>(g, a, G_min, st);
 }
 
 template <int XT>
 bq_status gemv_dispatch(const uint16_t *x, int M, int64_t K, const uint8_t *packed, const float *scales,
                         const uint8_t *zeros, const uint8_t *bit_map, int bits, int group, int64_t N, uint16_t *y,
                         cudaStream_t st) {
-  if (bit_map) {
-    Geom g = gemv_geometry(M, N, K, 128, true);
-    return launch_gemv_nb<XT, 4, 128, true>(g, x, M, K, packed, scales, zeros, bit_map, N, y, st);
-  }
-  const int64_t SU = group > tile_width(bits) ? group : tile_width(bits);
-  Geom g = gemv_geometry(M, N, K, SU, false);
-#define BQ_GV(B, G_)                                                                                 \
-  if (bits == B && group == G_)                                                                      \
-    return launch_gemv_nb<XT, B, G_, false>(g, x, M, K, packed, scales, zeros, nullptr, N, y, st);
+  GemvArgs a = {};
+  a.x = x;
+  a.packed = packed;
+  a.scales = scales;
+  a.zeros = zeros;
+  a.bit_map = bit_map;
+  a.y = y;
+  a.K = K;
+  a.N = N;
+  a.M = M;
+  if (bit_map) return launch_gemv_dispatch<XT, 4, 128, true>(a, st);
+#define BQ_GV(B, G_) \
+  if (bits == B && group == G_) return launch_gemv_dispatch<XT, B, G_, false>(a, st);
   BQ_GV(4, 128) BQ_GV(2, 64) BQ_GV(4, 32) BQ_GV(4, 64) BQ_GV(4, 256) BQ_GV(2, 32) BQ_GV(2, 128) BQ_GV(2, 256)
 #undef BQ_GV
   return BQ_ERR_UNSUPPORTED;
@@ -401,11 +435,10 @@ bq_status bq_linear(const void *x, bq_dtype xtype, int64_t M, int64_t K, const v
   if (xtype != BQ_F16 && xtype != BQ_BF16) return BQ_ERR_UNSUPPORTED;
   if (layout != BQ_LAYOUT_INTERLEAVED) return BQ_ERR_UNSUPPORTED;
   if (bit_map) {
-    if (N % 128 || K % 128) return BQ_ERR_SHAPE;
+    if (N % 128 || K % 512) return BQ_ERR_SHAPE;
   } else {
     if (!valid_bits(bits) || !linear_group_ok(bits, group)) return BQ_ERR_UNSUPPORTED;
-    const int64_t SU = group > tile_width(bits) ? group : tile_width(bits);
-    if (N % 16 || K % SU) return BQ_ERR_SHAPE;
+    if (N % 16 || K % (bits == 4 ? 256 : 512)) return BQ_ERR_SHAPE;
   }
   if (M == 0 || N == 0) return BQ_OK;
   if (!x || !y) return BQ_ERR_NULL;
@@ -414,7 +447,8 @@ bq_status bq_linear(const void *x, bq_dtype xtype, int64_t M, int64_t K, const v
     return cudaMemsetAsync(y, 0, (size_t)(M * N * 2), st) == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
   }
   if (!packed || !scales || !zeros) return BQ_ERR_NULL;
-  if (!aligned(x, 16) || !aligned(y, 16) || !aligned(packed, 16) || !aligned(scales, 4)) return BQ_ERR_ALIGN;
+  if (!aligned(x, 16) || !aligned(y, 16) || !aligned(packed, 16) || !aligned(scales, 16) || !aligned(zeros, 16))
+    return BQ_ERR_ALIGN;
   const uint16_t *xx = reinterpret_cast<const uint16_t *>(x);
   uint16_t *yy = reinterpret_cast<uint16_t *>(y);
   const uint8_t *pk = reinterpret_cast<const uint8_t *>(packed);
@@ -427,6 +461,32 @@ bq_status bq_linear(const void *x, bq_dtype xtype, int64_t M, int64_t K, const v
     if (s != BQ_OK) return s;
   }
   return BQ_OK;
+}
+
+bq_status bq_check_division(uint32_t s_bits_begin, uint32_t s_bits_end, int refinements,
+                            unsigned long long *result, void *stream) {
+  if (!result) return BQ_ERR_NULL;
+  if (s_bits_end <= s_bits_begin) return BQ_ERR_SHAPE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t grid = sm_count() * 8;
+  if (refinements == 1) check_division_kernel<1><<<grid, kThreads, 0, st>>>(s_bits_begin, s_bits_end, result);
+  else if (refinements == 2) check_division_kernel<2><<<grid, kThreads, 0, st>>>(s_bits_begin, s_bits_end, result);
+  else return BQ_ERR_UNSUPPORTED;
+  return launch_status();
+}
+
+bq_status bq_set_option(int option, int value) {
+  if (option == BQ_OPT_LINEAR_OVERLAP) {
+    if (value < 0 || value > 2) return BQ_ERR_UNSUPPORTED;
+    g_overlap_mode = value;
+    return BQ_OK;
+  }
+  return BQ_ERR_UNSUPPORTED;
+}
+
+int bq_get_option(int option) {
+  if (option == BQ_OPT_LINEAR_OVERLAP) return overlap_mode();
+  return -1;
 }
 
 bq_status bq_device_status(void *stream) {

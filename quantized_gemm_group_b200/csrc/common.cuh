@@ -64,6 +64,7 @@ template <> struct Elem<0> {  // fp16
     return *reinterpret_cast<uint32_t *>(&r);
   }
   static BQ_DEV uint16_t from_float(float v) { return __half_as_ushort(__float2half_rn(v)); }
+  static BQ_DEV float2 pair(uint32_t w) { return __half22float2(*reinterpret_cast<__half2 *>(&w)); }
 };
 template <> struct Elem<1> {  // bf16
   using T = __nv_bfloat16;
@@ -81,6 +82,7 @@ template <> struct Elem<1> {  // bf16
     return *reinterpret_cast<uint32_t *>(&r);
   }
   static BQ_DEV uint16_t from_float(float v) { return __bfloat16_as_ushort(__float2bfloat16_rn(v)); }
+  static BQ_DEV float2 pair(uint32_t w) { return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)); }
 };
 
 // NaN-propagating fp32 min / max.
@@ -136,25 +138,28 @@ struct GroupParams {
   int zc;        // z - kRoundMagicBits: added to the rounded bits of x/sd
   int z;         // zero point
   bool fast;     // 2^-60 <= sd <= 2^60: the refined division applies
+  bool clamp;    // some code of the group would reach 2^b (or the group is bad)
   bool bad;      // non-finite input or overflowing scale
 };
 
-BQ_DEV GroupParams group_params(float mn, float mx, int qmax) {
+template <int QMAX>
+BQ_DEV GroupParams group_params(float mn, float mx) {
   GroupParams p;
   p.bad = !(fabsf(mn) <= 3.402823466e38f) || !(fabsf(mx) <= 3.402823466e38f);
   float lo = fminf(mn, 0.0f);
   float hi = fmaxf(mx, 0.0f);
-  float s = __fdiv_rn(__fsub_rn(hi, lo), (float)qmax);
+  float s = __fdiv_rn(__fsub_rn(hi, lo), (float)QMAX);
   p.bad |= !(s <= 3.402823466e38f);
   if (p.bad || s == 0.0f) {
     // all-zero group: s = 0, z = 0 and every x is +-0, so x / 1 rounds to 0
-    // and every code is 0.  A bad group gets the same (unspecified) treatment.
+    // and every code is 0.  A bad group gets the same (unspecified) codes.
     p.s = 0.0f;
     p.sd = 1.0f;
     p.r = 1.0f;
     p.z = 0;
     p.zc = -kRoundMagicBits;
     p.fast = true;
+    p.clamp = true;
     return p;
   }
   p.s = s;
@@ -163,17 +168,107 @@ BQ_DEV GroupParams group_params(float mn, float mx, int qmax) {
   p.zc = p.z - kRoundMagicBits;
   p.fast = (s >= 8.67361738e-19f) && (s <= 1.15292150e18f);  // 2^-60 .. 2^60
   p.r = __frcp_rn(s);
+  // Codes are monotone in x, so only the largest element can overflow:
+  // round(hi / s) + z > 2^b - 1 decides whether this group needs the clamp.
+  p.clamp = __float2int_rn(__fdiv_rn(hi, s)) + p.z > QMAX;
   return p;
 }
 
-// Code of one element: min(round(x/s) + z, qmax).  round(x/s) + z >= 0 holds
-// for every x of the group (x >= lo gives round(x/s) >= round(lo/s) = -z), so
-// the unsigned min is the clamp; it also keeps a flagged bad group's garbage
-// inside its own field.  ALWAYS_FAST: fp16 inputs, whose scales always lie in
-// [2^-28, 2^16].
-template <int QMAX, bool ALWAYS_FAST>
-BQ_DEV uint32_t code_of(float x, const GroupParams &p) {
-  float t = (ALWAYS_FAST || p.fast) ? div_refined(x, p.sd, p.r) : __fdiv_rn(x, p.sd);
-  int q = __float_as_int(__fadd_rn(t, kRoundMagic)) + p.zc;
-  return min((uint32_t)q, (uint32_t)QMAX);
+// Codes of two elements of one group.
+// code = min(round(x/s) + z, 2^b - 1); round(x/s) + z >= 0 always holds
+// (x >= lo gives round(x/s) >= round(lo/s) = -z), and round(x/s) + z can
+// exceed 2^b - 1 only in groups flagged `clamp`.  The unsigned min also keeps
+// a bad group's garbage inside its own field.  ALWAYS_FAST: fp16 inputs,
+// whose scales always lie in [2^-28, 2^16].
+template <int QMAX, bool ALWAYS_FAST, bool CLAMP>
+BQ_DEV uint2 code_pair(float2 v, const GroupParams &p) {
+  float2 t;
+  if (ALWAYS_FAST || p.fast) {
+    const float2 r2 = make_float2(p.r, p.r), ns2 = make_float2(-p.sd, -p.sd);
+    float2 q0 = __fmul2_rn(v, r2);
+    float2 e0 = __ffma2_rn(ns2, q0, v);
+    float2 q1 = __ffma2_rn(e0, r2, q0);
+    float2 e1 = __ffma2_rn(ns2, q1, v);
+    t = __ffma2_rn(e1, r2, q1);
+  } else {
+    t = make_float2(__fdiv_rn(v.x, p.sd), __fdiv_rn(v.y, p.sd));
+  }
+  const float2 m = __fadd2_rn(t, make_float2(kRoundMagic, kRoundMagic));
+  uint32_t a = (uint32_t)(__float_as_int(m.x) + p.zc);
+  uint32_t b = (uint32_t)(__float_as_int(m.y) + p.zc);
+  if (CLAMP) {
+    a = min(a, (uint32_t)QMAX);
+    b = min(b, (uint32_t)QMAX);
+  }
+  return make_uint2(a, b);
 }
+
+// ---------------------------------------------------------------------------
+// interleaved layout addressing (see include/bq.h)
+// ---------------------------------------------------------------------------
+
+// 16-row tiles of a 128-row block (8, or fewer in the last partial block).
+BQ_DEV int64_t il_block_tiles(int64_t rt, int64_t N) {
+  const int64_t b = rt / 8;
+  const int64_t left = N / 16 - 8 * b;
+  return left < 8 ? left : 8;
+}
+// Byte offset of tile (global row tile rt, column block kt) of an N x K
+// matrix whose column blocks are T wide and hold BITS-bit codes.
+BQ_DEV int64_t il_tile_offset(int64_t rt, int64_t kt, int64_t N, int64_t K, int bits) {
+  const int64_t b = rt / 8;
+  return b * 128 * K * bits / 8 + (kt * il_block_tiles(rt, N) + rt % 8) * 512;
+}
+// Metadata index of group g of row n (G groups per row).
+BQ_DEV int64_t il_meta_index(int64_t n, int64_t g, int64_t N, int64_t G) {
+  const int64_t b = n / 128;
+  return 128 * G * b + g * (16 * il_block_tiles(n / 16, N)) + n % 128;
+}
+
+// ---------------------------------------------------------------------------
+// mbarrier / bulk-copy (TMA) helpers
+// ---------------------------------------------------------------------------
+
+BQ_DEV uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+BQ_DEV void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+BQ_DEV void mbar_fence_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+BQ_DEV void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+BQ_DEV void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+BQ_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait on the phase with the given parity: false after `limit` polls.
+constexpr uint32_t kWaitLimit = 1u << 22;
+BQ_DEV bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t limit = kWaitLimit) {
+  for (uint32_t i = 0; i < limit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+// One bulk copy global -> this CTA's shared memory, completing on `bar`.
+// dst, src 16-byte aligned; bytes a multiple of 16.
+BQ_DEV void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// Programmatic dependent launch: let the next kernel in the stream start
+// launching / wait until the previous one has completed and its memory is
+// visible.  Both are no-ops when the launch did not opt in.
+BQ_DEV void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+BQ_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }

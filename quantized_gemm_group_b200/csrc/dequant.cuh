@@ -38,17 +38,19 @@ __global__ void dequant_canonical_kernel(const uint8_t *__restrict__ packed, con
     dequant8_canonical<OT, BITS>(packed, scales, zeros, group, t * 8, out);
 }
 
-// interleaved: one warp per 512-byte tile; lane L owns rows r, r+8 and column
-// pairs (2c, 2c+1), (2c+8, 2c+9) of every 16-column run.
+// interleaved: one warp per 512-byte tile (logical row tile rt, column block
+// kt); lane L owns rows r, r+8 and column pairs (2c, 2c+1), (2c+8, 2c+9) of
+// every 16-column run.
 template <int OT, int BITS>
 BQ_DEV void dequant_tile(const uint8_t *__restrict__ packed, const float *__restrict__ scales,
-                         const uint8_t *__restrict__ zeros, int group, int64_t K, int64_t tile,
+                         const uint8_t *__restrict__ zeros, int group, int64_t N, int64_t K, int64_t tile,
                          int lane, typename OutT<OT>::T *__restrict__ out) {
   constexpr int T = (BITS == 4) ? 64 : 128;
   const int64_t kt_per_row = K / T;
-  const int64_t row0 = (tile / kt_per_row) * 16, col0 = (tile % kt_per_row) * T;
+  const int64_t rt = tile / kt_per_row, kt = tile % kt_per_row;
+  const int64_t row0 = rt * 16, col0 = kt * T;
   const int r = lane >> 2, c = lane & 3;
-  const uint4 v = *reinterpret_cast<const uint4 *>(packed + tile * 512 + lane * 16);
+  const uint4 v = *reinterpret_cast<const uint4 *>(packed + il_tile_offset(rt, kt, N, K, BITS) + lane * 16);
   const uint32_t words[4] = {v.x, v.y, v.z, v.w};
   const int64_t GK = K / group;
 #pragma unroll
@@ -64,8 +66,9 @@ BQ_DEV void dequant_tile(const uint8_t *__restrict__ packed, const float *__rest
       else { f_even = 4 * (run & 1) + slot; f_odd = f_even + 8; }
       const uint32_t mask = (1u << BITS) - 1;
       const uint32_t q0 = (w >> (BITS * f_even)) & mask, q1 = (w >> (BITS * f_odd)) & mask;
-      const float s = scales[row * GK + col / group];
-      const uint8_t z = zeros[row * GK + col / group];
+      const int64_t mi = il_meta_index(row, col / group, N, GK);
+      const float s = scales[mi];
+      const uint8_t z = zeros[mi];
       out[row * K + col] = OutT<OT>::cvt(deq(q0, z, s));
       out[row * K + col + 1] = OutT<OT>::cvt(deq(q1, z, s));
     }
@@ -81,7 +84,7 @@ __global__ void dequant_tiled_kernel(const uint8_t *__restrict__ packed, const f
   const int64_t tiles = (N / 16) * (K / T);
   for (int64_t t = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5; t < tiles;
        t += ((int64_t)gridDim.x * blockDim.x) >> 5)
-    dequant_tile<OT, BITS>(packed, scales, zeros, group, K, t, lane, out);
+    dequant_tile<OT, BITS>(packed, scales, zeros, group, N, K, t, lane, out);
 }
 
 // mixed: one warp per 512-byte tile of either width; a 128-row block holds
@@ -106,8 +109,8 @@ __global__ void dequant_mixed_kernel(const uint8_t *__restrict__ packed, const f
     if (TILED) {
       const int64_t tiles = 8 * K / (bits == 4 ? 64 : 128);
       for (int64_t t = 0; t < tiles; ++t) {
-        if (bits == 4) dequant_tile<OT, 4>(pk, sc, ze, 128, K, t, lane, o);
-        else dequant_tile<OT, 2>(pk, sc, ze, 64, K, t, lane, o);
+        if (bits == 4) dequant_tile<OT, 4>(pk, sc, ze, 128, 128, K, t, lane, o);
+        else dequant_tile<OT, 2>(pk, sc, ze, 64, 128, K, t, lane, o);
       }
     } else {
       for (int64_t e = lane * 8; e < 128 * K; e += 256) {

@@ -1,30 +1,43 @@
 // gemv.cuh -- decode-path weight-only linear, M <= 16 tokens:
 //   y[m, n] = sum_g s[n, g] * sum_{k in g} x[m, k] * (q[n, k] - z[n, g])
 // ("A Survey of Low-bit Large Language Models", section 6.2: weight-only
-// quantization dequantizes and runs a 16-bit matmul, and gains by moving
+// quantization dequantizes and runs a 16-bit matmul and gains by moving
 // fewer bytes; "大模型量化实战" section 3.3: dequantize and multiply inside one
 // kernel so no intermediate goes back to memory).
 //
-// Design (HBM-bound; the weights are read exactly once):
-//  * Codes use the interleaved layout: lane L's 16-byte slot of a 512-byte
-//    tile is, word by word, the A operand of a 16x8x16 bf16 mma.sync for
-//    rows (L/4, L/4+8) of the 16-row tile.  One LOP3 per register builds
-//    (128 + q) pairs as bf16x2 (magic exponent 0x4300), one HSUB2 removes
-//    (128 + z): the operand is the exact integer q - z.
-//  * x^T is the B operand (8 tokens per mma; two mmas for M > 8).  A CTA
-//    stages its K-slice of x once in shared memory (rows padded by 16 bytes
-//    so ldmatrix is conflict-free) and reads fragments with ldmatrix.x4.
-//  * Each group's products accumulate in fp32 from zero; the group's fp32
-//    scale is then applied per row in an FMA into the running sum.
-//  * A CTA covers 16*R rows and a K-slice; its warps split that slice
-//    further; warp partials meet in shared memory.  CTAs that split K form a
-//    thread-block cluster and the partials are reduced through distributed
-//    shared memory in fixed rank order: deterministic, no global scratch.
-//  * Tile loads for the next super-unit are issued before the current one is
-//    computed (register double buffering).
+// Design (HBM-bound; every weight byte is read exactly once):
+//  * A CTA owns one 128-row block (8 row tiles of 16; fewer in a last partial
+//    block) and a K-slice of KC columns.  In the interleaved layout the codes
+//    of a whole block for a run of column blocks are contiguous, and so are
+//    its scales and its zeros for a run of groups.  One producer warp stages
+//    the block's scales and zeros for the slice and the slice of x once (x
+//    rows padded by 16 bytes so ldmatrix is conflict-free; padding tokens read
+//    a 16-byte zero chunk), and streams the codes through a shared-memory ring
+//    of 16 KB stages, one bulk asynchronous copy per stage (cp.async.bulk
+//    completing on an mbarrier with a transaction count).  Bulk copies reach
+//    full HBM bandwidth only when they are large (measured on B200: ~1.5-3
+//    TB/s with 2 KB copies, 6.5-7 TB/s with 16-32 KB copies), hence this
+//    layout.
+//  * Consumer warp j reads its lane's 16-byte slot of row tile j in each
+//    column block (conflict-free), builds exact (q - z) operands in registers
+//    (one LOP3 against the 0x4300 bf16 magic exponent plus one bf16x2
+//    subtract per register) and issues m16n8k16 mma.sync with x^T as the B
+//    operand.  Each group accumulates in fp32 from zero; the group's fp32
+//    scale is applied per row in an FMA into the running sum.
+//  * CTAs splitting K form a thread-block cluster; each pushes its partial
+//    sums into the owning rank's shared memory (distributed shared memory),
+//    one cluster barrier publishes them, and each rank sums its slice in
+//    fixed rank order: deterministic, no global scratch.  Without a split the
+//    consumers write y directly.
+//  * Programmatic dependent launch (opt-in): the kernel lets the next kernel
+//    launch early and, when the caller guarantees that the weights are not
+//    written by the preceding kernel, starts streaming weights before waiting
+//    for it; x is always read after the wait.
+//  * Every mbarrier wait is bounded; on expiry the kernel records
+//    BQ_FLAG_TIMEOUT, stops issuing copies, waits (bounded) for the copies it
+//    already issued, and still joins the cluster barriers.
 #pragma once
 #include <cooperative_groups.h>
-#include <type_traits>
 
 #include "common.cuh"
 
@@ -34,13 +47,15 @@ namespace cg = cooperative_groups;
 template <int XT> struct MmaT;
 template <> struct MmaT<1> {  // bf16
   static constexpr uint32_t kMagic = 0x43004300u;  // bf16x2 (128, 128)
+  static constexpr uint32_t kOne2 = 0x3F803F80u;   // bf16x2 (1, 1)
   static BQ_DEV uint32_t zpair(uint32_t z) {     // bf16x2 (128 + z, 128 + z), exact
     uint32_t h = 0x4300u | z;
     return h | (h << 16);
   }
   static BQ_DEV uint32_t sub2(uint32_t a, uint32_t b) {
-    __nv_bfloat162 r = __hsub2(*reinterpret_cast<__nv_bfloat162 *>(&a), *reinterpret_cast<__nv_bfloat162 *>(&b));
-    return *reinterpret_cast<uint32_t *>(&r);
+    uint32_t r;
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
   }
   static BQ_DEV void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -53,13 +68,15 @@ template <> struct MmaT<1> {  // bf16
 };
 template <> struct MmaT<0> {  // fp16
   static constexpr uint32_t kMagic = 0x64006400u;  // fp16x2 (1024, 1024)
+  static constexpr uint32_t kOne2 = 0x3C003C00u;   // fp16x2 (1, 1)
   static BQ_DEV uint32_t zpair(uint32_t z) {
     uint32_t h = 0x6400u | z;
     return h | (h << 16);
   }
   static BQ_DEV uint32_t sub2(uint32_t a, uint32_t b) {
-    __half2 r = __hsub2(*reinterpret_cast<__half2 *>(&a), *reinterpret_cast<__half2 *>(&b));
-    return *reinterpret_cast<uint32_t *>(&r);
+    uint32_t r;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
   }
   static BQ_DEV void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -83,198 +100,314 @@ BQ_DEV void ldmatrix_x4(uint32_t (&r)[4], uint32_t smem_addr) {
                : "r"(smem_addr));
 }
 
-// Shared-memory layout (dynamic), CTA = NWR x NWK warps covering
-// ROWS = 16 * R * NWR rows and KC = NWK * KW columns:
-//   xs   [8*NB][KC + 8] activations (16-bit), rows padded by 16 bytes
-//   red  [NWK][8*NB][ROWS] fp32 partials of the K-slices (token-major)
-//   part [8*NB][ROWS] fp32 CTA partial (token-major), read by the cluster
-inline size_t gemv_smem_bytes(int NB, int R, int NWR, int NWK, int64_t KC) {
-  const size_t tok = 8 * NB, rows = 16 * R * NWR;
-  return tok * (KC + 8) * 2 + (size_t)NWK * tok * rows * 4 + tok * rows * 4;
+BQ_DEV uint4 lds_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
 }
 
-// Body of one warp over its K range for the CTA's R row tiles.  `pk`, `sc`,
-// `ze` address the matrix (or the mixed block) the rows belong to; `row0` is
-// the first row relative to them and `kw0` the warp's first column.
-template <int XT, int BITS, int G, int NB, int R>
-BQ_DEV void gemv_warp(const uint8_t *__restrict__ pk, const float *__restrict__ sc,
-                      const uint8_t *__restrict__ ze, int64_t K, int64_t row0, int64_t kw0, int64_t KW,
-                      int64_t kc0, uint32_t xs_base, int xs_stride_bytes, int lane, float (&acc)[R][NB][4]) {
-  using MT = MmaT<XT>;
-  constexpr int T = (BITS == 4) ? 64 : 128;       // tile width
-  constexpr int SU = (G > T) ? G : T;              // super-unit width
-  constexpr int TILES = SU / T;
-  constexpr int STEPS_PER_G = G / 16;
-  constexpr int GROUPS = SU / G;
-  constexpr uint32_t MASK = (BITS == 4) ? 0x000F000Fu : 0x00030003u;
-  const int r = lane >> 2;
-  const int64_t GK = K / G;
-  const int64_t KT = K / T;
+constexpr int kGemvMaxStages = 4;
+constexpr int kGemvMaxConsumers = 8;
 
-  // ldmatrix row address of this lane: token lane%8 (+8 for the second
-  // block), column offset 8*(lane/8) inside a pair of k16 steps.
-  const uint32_t xs_lane = xs_base + (uint32_t)((lane & 7) * xs_stride_bytes + (lane >> 3) * 16);
+// Per-width stage geometry: a stage is SC columns of a full 128-row block,
+// 16 KB of packed codes for either width (SC = 256 at 4 bits, 512 at 2 bits).
+template <int BITS, int G> struct StageG {
+  static constexpr int T = (BITS == 4) ? 64 : 128;   // tile width
+  static constexpr int SC = (BITS == 4) ? 256 : 512;  // columns per stage
+  static constexpr int TPS = SC / T;                  // column blocks per stage (4)
+  static constexpr int GPS = SC / G;                  // groups per stage
+  static constexpr int STEPS_PER_G = G / 16;
+  static constexpr int W_BYTES = TPS * 8 * 512;       // packed codes of the block (16 KB)
+  static_assert(SC % G == 0 && STEPS_PER_G % 2 == 0, "bad stage geometry");
+};
 
-  const int nsu = (int)(KW / SU);
-  uint4 buf[2][R][TILES];
-  uint32_t zb[2][R][GROUPS][2];
-  float sb[2][R][GROUPS][2];
+// Shared-memory layout (bytes), all staged per CTA:
+//   x     [M][KC + 8] 16-bit rows (only the real tokens), then a 16-byte
+//         zero chunk that ldmatrix reads for padding tokens
+//   meta  scales [KC/G][rows] fp32 then zeros [KC/G][rows] u8 of the block
+//   ring  `stages` x 16 KB of packed codes
+//   part  split-K receive buffer: S_k slices of ceil(TOK * rows / S_k) fp32
+//   bars  full[stages], empty[stages], x/meta barrier, abort flag
+struct GemvSmem {
+  int zero_off, s_off, z_off, ring_off, part_off, bar_off, total;
+};
 
-  auto load_su = [&](int i, auto slot_c) {
-    constexpr int slot = decltype(slot_c)::value;
-    const int64_t col = kw0 + (int64_t)i * SU;
-#pragma unroll
-    for (int rb = 0; rb < R; ++rb) {
-      const int64_t rt = row0 / 16 + rb;
-#pragma unroll
-      for (int t = 0; t < TILES; ++t)
-        buf[slot][rb][t] = ld_stream_v4(pk + (rt * KT + col / T + t) * 512 + lane * 16);
-#pragma unroll
-      for (int gi = 0; gi < GROUPS; ++gi)
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int64_t idx = (row0 + rb * 16 + r + 8 * h) * GK + col / G + gi;
-          sb[slot][rb][gi][h] = __ldg(sc + idx);
-          zb[slot][rb][gi][h] = __ldg(ze + idx);
-        }
-    }
+inline GemvSmem gemv_smem_layout(int M, int TOK, int64_t KC, int groups, int stages) {
+  GemvSmem L;
+  L.zero_off = (int)(M * (KC + 8) * 2);
+  L.s_off = (L.zero_off + 16 + 127) / 128 * 128;
+  L.z_off = L.s_off + groups * 128 * 4;
+  L.ring_off = (L.z_off + groups * 128 + 127) / 128 * 128;
+  L.part_off = L.ring_off + stages * 16384;
+  L.bar_off = L.part_off + (TOK * 128 + 8) * 4;
+  L.total = L.bar_off + (2 * stages + 1) * 8 + 16;
+  return L;
+}
+
+struct GemvArgs {
+  const uint16_t *x;
+  const uint8_t *packed;
+  const float *scales;
+  const uint8_t *zeros;
+  const uint8_t *bit_map;
+  uint16_t *y;
+  int64_t K, N, KC;
+  int M;
+  int stages;
+  int prefetch_before_wait;  // weights may be streamed before the programmatic wait
+  GemvSmem L;
+};
+
+// Producer warp.  Streams the CTA's K-slice of its 128-row block through the
+// ring, one 16 KB bulk copy per stage (contiguous in the interleaved layout),
+// after lane 0 armed the stage's full barrier; stages the block's scales and
+// zeros for the slice (two copies, contiguous in the interleaved metadata
+// layout) and its x rows (one copy per token) once, on the x/meta barrier.
+// `pk`, `sc`, `ze` point at the block's first byte / element; `R` = row tiles.
+template <int BITS, int G>
+BQ_DEV void gemv_produce(const GemvArgs &a, const uint8_t *pk, const float *sc, const uint8_t *ze, int R,
+                         int64_t kc0, uint32_t smem, uint32_t bars, volatile int *abort, int lane) {
+  using SG = StageG<BITS, G>;
+  const int n = (int)(a.KC / SG::SC);
+  const int S = a.stages;
+  const int rows = 16 * R;
+  const uint32_t wb = (uint32_t)(SG::TPS * R * 512);
+  const uint32_t xm_full = bars + 8u * (2 * S);
+  const int groups = (int)(a.KC / G);
+  auto issue = [&](int i, uint32_t full) {
+    const uint32_t st = smem + (uint32_t)(a.L.ring_off + (i % S) * 16384);
+    const int64_t ks = kc0 + (int64_t)i * SG::SC;
+    bulk_g2s(st, pk + (ks / SG::T) * R * 512, wb, full);
   };
+  auto stage_meta = [&]() {  // arms the x/meta barrier for metadata and x
+    if (lane == 0) {
+      mbar_arrive_expect_tx(xm_full, (uint32_t)(groups * rows * 5 + a.M * a.KC * 2));
+      bulk_g2s(smem + a.L.s_off, sc + (kc0 / G) * rows, (uint32_t)(groups * rows * 4), xm_full);
+      bulk_g2s(smem + a.L.z_off, ze + (kc0 / G) * rows, (uint32_t)(groups * rows), xm_full);
+    }
+    __syncwarp();
+  };
+  auto stage_x = [&]() {
+    for (int m = lane; m < a.M; m += 32)
+      bulk_g2s(smem + (uint32_t)(m * (a.KC + 8) * 2), a.x + m * a.K + kc0, (uint32_t)(a.KC * 2), xm_full);
+  };
+  const int pre = n < S ? n : S;
+  if (!a.prefetch_before_wait) pdl_wait();
+  stage_meta();
+  for (int i = 0; i < pre; ++i) {
+    const uint32_t full = bars + 8u * i;
+    if (lane == 0) {
+      mbar_arrive_expect_tx(full, wb);
+      issue(i, full);
+    }
+  }
+  if (a.prefetch_before_wait) pdl_wait();
+  stage_x();
+  int issued = pre;
+  int slot = pre % S, phase = (pre / S) & 1;
+  for (int i = pre; i < n; ++i) {
+    const uint32_t full = bars + 8u * slot, empty = bars + 8u * (S + slot);
+    const bool ok = __all_sync(0xffffffffu, (*abort == 0) && mbar_wait(empty, phase ^ 1));
+    if (!ok) {
+      if (lane == 0) {
+        *abort = 1;
+        bq_flag(BQ_FLAG_TIMEOUT);
+      }
+      break;
+    }
+    if (lane == 0) {
+      mbar_arrive_expect_tx(full, wb);
+      issue(i, full);
+    }
+    issued = i + 1;
+    if (++slot == S) {
+      slot = 0;
+      phase ^= 1;
+    }
+  }
+  __syncwarp();
+  if (*abort && lane == 0) {
+    // let the copies already issued land before the CTA can exit
+    mbar_wait(xm_full, 0);
+    for (int i = (issued > S ? issued - S : 0); i < issued; ++i) mbar_wait(bars + 8u * (i % S), (i / S) & 1);
+  }
+}
 
-  auto compute_su = [&](int i, auto slot_c) {
-    constexpr int slot = decltype(slot_c)::value;
-    const int64_t col_in_cta = kw0 - kc0 + (int64_t)i * SU;
+// Consumer warp j: 16-row tile j of the CTA's block over the whole K-slice.
+template <int XT, int BITS, int G, int NB>
+BQ_DEV void gemv_consume(const GemvArgs &a, int j, int R, uint32_t smem, uint32_t bars, volatile int *abort,
+                         int lane, float (&acc)[NB][4]) {
+  using MT = MmaT<XT>;
+  using SG = StageG<BITS, G>;
+  constexpr uint32_t MASK = (BITS == 4) ? 0x000F000Fu : 0x00030003u;
+  const int n = (int)(a.KC / SG::SC);
+  const int S = a.stages;
+  const int rows = 16 * R;
+  const int r = lane >> 2;
+  const int xstride = (int)(a.KC + 8) * 2;
+  // ldmatrix row address of this lane for token block nb: token (lane & 7) +
+  // 8 nb, column offset 8 (lane / 8) inside a pair of k16 steps; tokens >= M
+  // read the zero chunk (and do not advance with k)
+  uint32_t x_lane[NB];
+  uint32_t x_step[NB];
 #pragma unroll
-    for (int gi = 0; gi < GROUPS; ++gi) {
-      float c[R][NB][4];
-      uint32_t zz[R][2];
+  for (int nb = 0; nb < NB; ++nb) {
+    const int tok = (lane & 7) + 8 * nb;
+    const bool real = tok < a.M;
+    x_lane[nb] = real ? smem + (uint32_t)(tok * xstride + (lane >> 3) * 16) : smem + a.L.zero_off;
+    x_step[nb] = real ? 1u : 0u;
+  }
+  if (*abort || !mbar_wait(bars + 8u * (2 * S), 0)) {  // x and metadata staged
+    *abort = 1;
+    bq_flag(BQ_FLAG_TIMEOUT);
+    return;
+  }
+  const uint32_t stile = smem + a.L.s_off + (j * 16 + r) * 4;
+  const uint32_t ztile = smem + a.L.z_off + j * 16 + r;
+  int slot = 0, phase = 0;
+  for (int i = 0; i < n; ++i) {
+    const uint32_t full = bars + 8u * slot, empty = bars + 8u * (S + slot);
+    if (*abort || !mbar_wait(full, phase)) {
+      *abort = 1;
+      bq_flag(BQ_FLAG_TIMEOUT);
+      break;
+    }
+    const uint32_t wt = smem + (uint32_t)(a.L.ring_off + slot * 16384) + j * 512 + lane * 16;
+    uint4 tiles[SG::TPS];
 #pragma unroll
-      for (int rb = 0; rb < R; ++rb) {
-        zz[rb][0] = MT::zpair(zb[slot][rb][gi][0]);
-        zz[rb][1] = MT::zpair(zb[slot][rb][gi][1]);
+    for (int t = 0; t < SG::TPS; ++t) tiles[t] = lds_v4(wt + t * R * 512);
+    // the stage's codes are in registers now: hand the slot back to the
+    // producer before computing, so the ring keeps prefetching
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty);
+    if (++slot == S) {
+      slot = 0;
+      phase ^= 1;
+    }
+#pragma unroll
+    for (int gi = 0; gi < SG::GPS; ++gi) {
+      const int g = i * SG::GPS + gi;  // group within the CTA's slice
+      float s0, s1;
+      uint32_t z0, z1;
+      asm volatile("ld.shared.f32 %0, [%1];" : "=f"(s0) : "r"(stile + g * rows * 4));
+      asm volatile("ld.shared.f32 %0, [%1];" : "=f"(s1) : "r"(stile + (g * rows + 8) * 4));
+      asm volatile("ld.shared.u8 %0, [%1];" : "=r"(z0) : "r"(ztile + g * rows));
+      asm volatile("ld.shared.u8 %0, [%1];" : "=r"(z1) : "r"(ztile + g * rows + 8));
+      // bf16 with at most 8 tokens: the operands are the exact integers
+      // 128 + q (magic exponent 0x4300), so y_group = s * (sum x (128 + q) -
+      // (128 + z) sum x), the x sums of each token coming from one extra mma
+      // against all-ones.  Otherwise (fp16: base 1024, larger cancellation;
+      // 16 tokens: the extra mma would double the tensor work) exact (q - z)
+      // operands from one 16-bit-pair subtract per register.
+      constexpr bool kOnes = (XT == 1 && NB == 1);
+      const uint32_t zz0 = MT::zpair(z0), zz1 = MT::zpair(z1);
+      const float zf0 = kOnes ? (float)(128 + (int)z0) : 0.0f, zf1 = kOnes ? (float)(128 + (int)z1) : 0.0f;
+      float c[2][NB][4], cx[NB][4];
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
-          for (int j = 0; j < 4; ++j) c[rb][nb][j] = 0.0f;
-      }
+          for (int q = 0; q < 4; ++q) c[h][nb][q] = 0.0f;
 #pragma unroll
-      for (int sp = 0; sp < STEPS_PER_G; sp += 2) {  // pairs of k16 steps
-        const int step0 = gi * STEPS_PER_G + sp;
+      for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) cx[nb][q] = 0.0f;
+#pragma unroll
+      for (int sp = 0; sp < SG::STEPS_PER_G; sp += 2) {
+        const int step0 = gi * SG::STEPS_PER_G + sp;               // k16 step within the stage
+        const uint32_t kbytes = (uint32_t)((i * SG::SC + step0 * 16) * 2);  // column offset in x rows
         uint32_t bfr[NB][4];
 #pragma unroll
-        for (int nb = 0; nb < NB; ++nb)
-          ldmatrix_x4(bfr[nb], xs_lane + (uint32_t)(nb * 8 * xs_stride_bytes) +
-                                   (uint32_t)((col_in_cta + step0 * 16) * 2));
+        for (int nb = 0; nb < NB; ++nb) ldmatrix_x4(bfr[nb], x_lane[nb] + x_step[nb] * kbytes);
 #pragma unroll
         for (int ss = 0; ss < 2; ++ss) {
           const int step = step0 + ss;
-          const int t = step / (T / 16);    // tile within the super-unit
-          const int run = step % (T / 16);  // 16-column run within the tile
+          const int t = step / (SG::T / 16);
+          const int run = step % (SG::T / 16);
+          const uint32_t words[4] = {tiles[t].x, tiles[t].y, tiles[t].z, tiles[t].w};
+          const uint32_t w = words[BITS == 4 ? run : run / 2];
+          const int base = (BITS == 4) ? 0 : 4 * (run & 1);
+          uint32_t av[4];
 #pragma unroll
-          for (int rb = 0; rb < R; ++rb) {
-            const uint4 v = buf[slot][rb][t];
-            const uint32_t words[4] = {v.x, v.y, v.z, v.w};
-            const uint32_t w = words[BITS == 4 ? run : run / 2];
-            const int base = (BITS == 4) ? 0 : 4 * (run & 1);
-            uint32_t a[4];
+          for (int si = 0; si < 4; ++si) {
+            av[si] = and_or(w >> (BITS * (base + si)), MASK, MT::kMagic);
+            if (!kOnes) av[si] = MT::sub2(av[si], (si & 1) ? zz1 : zz0);
+          }
 #pragma unroll
-            for (int si = 0; si < 4; ++si) {
-              const uint32_t p = and_or(w >> (BITS * (base + si)), MASK, MT::kMagic);
-              a[si] = MT::sub2(p, zz[rb][si & 1]);
+          for (int nb = 0; nb < NB; ++nb) {
+            MT::mma(c[ss][nb], av, bfr[nb][2 * ss], bfr[nb][2 * ss + 1]);
+            if (kOnes) {
+              const uint32_t ones[4] = {MT::kOne2, MT::kOne2, MT::kOne2, MT::kOne2};
+              MT::mma(cx[nb], ones, bfr[nb][2 * ss], bfr[nb][2 * ss + 1]);
             }
-#pragma unroll
-            for (int nb = 0; nb < NB; ++nb) MT::mma(c[rb][nb], a, bfr[nb][2 * ss], bfr[nb][2 * ss + 1]);
           }
         }
       }
 #pragma unroll
-      for (int rb = 0; rb < R; ++rb) {
-        const float s0 = sb[slot][rb][gi][0], s1 = sb[slot][rb][gi][1];
-#pragma unroll
-        for (int nb = 0; nb < NB; ++nb) {
-          acc[rb][nb][0] = __fmaf_rn(s0, c[rb][nb][0], acc[rb][nb][0]);
-          acc[rb][nb][1] = __fmaf_rn(s0, c[rb][nb][1], acc[rb][nb][1]);
-          acc[rb][nb][2] = __fmaf_rn(s1, c[rb][nb][2], acc[rb][nb][2]);
-          acc[rb][nb][3] = __fmaf_rn(s1, c[rb][nb][3], acc[rb][nb][3]);
-        }
+      for (int nb = 0; nb < NB; ++nb) {
+        acc[nb][0] = __fmaf_rn(s0, __fmaf_rn(-zf0, cx[nb][0], c[0][nb][0] + c[1][nb][0]), acc[nb][0]);
+        acc[nb][1] = __fmaf_rn(s0, __fmaf_rn(-zf0, cx[nb][1], c[0][nb][1] + c[1][nb][1]), acc[nb][1]);
+        acc[nb][2] = __fmaf_rn(s1, __fmaf_rn(-zf1, cx[nb][2], c[0][nb][2] + c[1][nb][2]), acc[nb][2]);
+        acc[nb][3] = __fmaf_rn(s1, __fmaf_rn(-zf1, cx[nb][3], c[0][nb][3] + c[1][nb][3]), acc[nb][3]);
       }
-    }
-  };
-
-  using S0 = std::integral_constant<int, 0>;
-  using S1 = std::integral_constant<int, 1>;
-  if (nsu > 0) load_su(0, S0{});
-  for (int i = 0; i < nsu; i += 2) {
-    if (i + 1 < nsu) load_su(i + 1, S1{});
-    compute_su(i, S0{});
-    if (i + 1 < nsu) {
-      if (i + 2 < nsu) load_su(i + 2, S0{});
-      compute_su(i + 1, S1{});
     }
   }
 }
 
-// Kernel.  grid = (N / ROWS, S); cluster = (1, S, 1); block = NWR * NWK
-// warps.  Warp w covers rows 16 R (w % NWR) .. of the CTA and the K-slice
-// w / NWR.  bit_map == nullptr: uniform BITS / G.  Otherwise one width per
-// 128-row block (ROWS divides 128) and the CTA runs (4, 128) or (2, 64).
-template <int XT, int BITS, int G, int NB, int R, bool MIXED>
-__global__ void __launch_bounds__(256)
-gemv_kernel(const uint16_t *__restrict__ x, int M, int64_t K, const uint8_t *__restrict__ packed,
-            const float *__restrict__ scales, const uint8_t *__restrict__ zeros,
-            const uint8_t *__restrict__ bit_map, int64_t N, uint16_t *__restrict__ y, int64_t KC, int64_t KW,
-            int NWR) {
+// Kernel.  grid = (ceil(N / 128), S_k); cluster = (1, S_k, 1); block = 9
+// warps (8 consumers, one per 16-row tile of the block; warp 8 produces).
+// bit_map == nullptr: uniform BITS / G.  Otherwise one width per 128-row
+// block and the CTA runs (4, 128) or (2, 64).
+template <int XT, int BITS, int G, int NB, bool MIXED>
+__global__ void __launch_bounds__(32 * (kGemvMaxConsumers + 1), 2)
+gemv_kernel(const GemvArgs a) {
   using MT = MmaT<XT>;
-  extern __shared__ __align__(16) unsigned char smem[];
-  const int NW = blockDim.x >> 5;
-  const int NWK = NW / NWR;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int wr = warp % NWR, wk = warp / NWR;
-  cg::cluster_group cluster = cg::this_cluster();
-  const int S = (int)cluster.dim_blocks().y;
-  const int rank = (int)cluster.block_rank();
   constexpr int TOK = 8 * NB;
-  const int ROWS = 16 * R * NWR;
-  const int64_t kc0 = (int64_t)blockIdx.y * KC;
-  const int64_t row0 = (int64_t)blockIdx.x * ROWS;
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int NC = kGemvMaxConsumers;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int SK = (int)cluster.dim_blocks().y;
+  const int rank = (int)cluster.block_rank();
+  const int64_t kc0 = (int64_t)blockIdx.y * a.KC;
+  const int64_t blk = blockIdx.x;
+  const int64_t row0 = blk * 128;
+  const int R = (int)((a.N - row0) / 16 < 8 ? (a.N - row0) / 16 : 8);  // row tiles in the block
+  const int ROWS = 16 * R;
+  const uint32_t smem = smem_u32(smem_raw);
+  const uint32_t bars = smem + a.L.bar_off;
+  volatile int *abort = reinterpret_cast<volatile int *>(smem_raw + a.L.bar_off + (2 * a.stages + 1) * 8);
+  float *part = reinterpret_cast<float *>(smem_raw + a.L.part_off);
 
-  uint16_t *xs = reinterpret_cast<uint16_t *>(smem);
-  const int xs_stride = (int)(KC + 8);  // elements
-  float *red = reinterpret_cast<float *>(smem + (size_t)TOK * xs_stride * 2);
-  float *part = red + (size_t)NWK * TOK * ROWS;
+  pdl_launch_dependents();
 
-  // Wait for the previous kernel in the stream before touching x or y
-  // (programmatic dependent launch; a no-op otherwise).
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-
-  // stage x[:, kc0 : kc0 + KC] (token rows >= M are zero)
-  const int64_t chunks_per_row = KC / 8;
-  for (int64_t i = threadIdx.x; i < TOK * chunks_per_row; i += blockDim.x) {
-    const int m = (int)(i / chunks_per_row);
-    const int64_t ch = i - m * chunks_per_row;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (m < M) v = *reinterpret_cast<const uint4 *>(x + (int64_t)m * K + kc0 + ch * 8);
-    *reinterpret_cast<uint4 *>(xs + (int64_t)m * xs_stride + ch * 8) = v;
+  // the zero chunk read by padding tokens
+  if (threadIdx.x == 0) *reinterpret_cast<uint4 *>(smem_raw + a.L.zero_off) = make_uint4(0, 0, 0, 0);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < a.stages; ++s) {
+      mbar_init(bars + 8u * s, 1);
+      mbar_init(bars + 8u * (a.stages + s), R);
+    }
+    mbar_init(bars + 8u * (2 * a.stages), 1);
+    *abort = 0;
+    mbar_fence_init();
   }
   __syncthreads();
 
-  float acc[R][NB][4];
-#pragma unroll
-  for (int rb = 0; rb < R; ++rb)
-#pragma unroll
-    for (int nb = 0; nb < NB; ++nb)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) acc[rb][nb][j] = 0.0f;
-
-  const uint32_t xs_base = (uint32_t)__cvta_generic_to_shared(xs);
-  const int64_t kw0 = kc0 + (int64_t)wk * KW;
-  const int64_t wrow0 = row0 + (int64_t)wr * 16 * R;
+  // width of this block and where its codes / metadata start
+  int bits = BITS;
+  const uint8_t *pk;
+  const float *sc;
+  const uint8_t *ze;
   if (!MIXED) {
-    gemv_warp<XT, BITS, G, NB, R>(packed, scales, zeros, K, wrow0, kw0, KW, kc0, xs_base, xs_stride * 2, lane, acc);
+    pk = a.packed + blk * 128 * a.K * BITS / 8;
+    sc = a.scales + blk * 128 * (a.K / G);
+    ze = a.zeros + blk * 128 * (a.K / G);
   } else {
-    const int64_t blk = row0 / 128;
     int64_t sb = 0, sg = 0;
-    for (int64_t j = lane; j < blk; j += 32) {
-      const int b = bit_map[j];
+    for (int64_t jb = lane; jb < blk; jb += 32) {
+      const int b = a.bit_map[jb];
       sb += b;
       sg += (b == 4) ? 1 : 2;
     }
@@ -283,55 +416,80 @@ gemv_kernel(const uint16_t *__restrict__ x, int M, int64_t K, const uint8_t *__r
       sb += __shfl_xor_sync(0xffffffffu, sb, off);
       sg += __shfl_xor_sync(0xffffffffu, sg, off);
     }
-    const uint8_t *pk = packed + sb * 16 * K;
-    const float *sc = scales + sg * K;
-    const uint8_t *ze = zeros + sg * K;
-    const int bits = bit_map[blk];
-    const int64_t rr0 = wrow0 - blk * 128;
-    if (bits == 4) {
-      gemv_warp<XT, 4, 128, NB, R>(pk, sc, ze, K, rr0, kw0, KW, kc0, xs_base, xs_stride * 2, lane, acc);
-    } else if (bits == 2) {
-      gemv_warp<XT, 2, 64, NB, R>(pk, sc, ze, K, rr0, kw0, KW, kc0, xs_base, xs_stride * 2, lane, acc);
-    } else if (lane == 0) {
-      bq_flag(BQ_FLAG_BADMAP);
+    pk = a.packed + sb * 16 * a.K;
+    sc = a.scales + sg * a.K;
+    ze = a.zeros + sg * a.K;
+    bits = a.bit_map[blk];
+    if (bits != 4 && bits != 2) {
+      if (threadIdx.x == 0) bq_flag(BQ_FLAG_BADMAP);
+      bits = 0;
     }
   }
 
-  // warp partials -> shared (token-major), one slice per K-slice wk
-  {
-    const int r = lane >> 2, c = lane & 3;
-    float *w = red + (size_t)wk * TOK * ROWS;
+  float acc[NB][4];
 #pragma unroll
-    for (int rb = 0; rb < R; ++rb)
+  for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) acc[nb][q] = 0.0f;
+
+  if (warp == NC) {
+    if (bits != 0) {
+      if (!MIXED) gemv_produce<BITS, G>(a, pk, sc, ze, R, kc0, smem, bars, abort, lane);
+      else if (bits == 4) gemv_produce<4, 128>(a, pk, sc, ze, R, kc0, smem, bars, abort, lane);
+      else gemv_produce<2, 64>(a, pk, sc, ze, R, kc0, smem, bars, abort, lane);
+    }
+  } else if (bits != 0 && warp < R) {
+    if (!MIXED) gemv_consume<XT, BITS, G, NB>(a, warp, R, smem, bars, abort, lane, acc);
+    else if (bits == 4) gemv_consume<XT, 4, 128, NB>(a, warp, R, smem, bars, abort, lane, acc);
+    else gemv_consume<XT, 2, 64, NB>(a, warp, R, smem, bars, abort, lane, acc);
+  }
+
+  if (SK == 1) {
+    // no split: every consumer writes its own rows and tokens
+    pdl_wait();  // y may be read by the previous kernel: write only after it completed
+    if (warp < R) {
+      const int r = lane >> 2, c = lane & 3;
 #pragma unroll
       for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int row = wr * 16 * R + rb * 16 + r + 8 * (j >> 1);
-          const int tok = nb * 8 + 2 * c + (j & 1);
-          w[tok * ROWS + row] = acc[rb][nb][j];
+        for (int q = 0; q < 4; ++q) {
+          const int row = warp * 16 + r + 8 * (q >> 1);
+          const int tok = nb * 8 + 2 * c + (q & 1);
+          if (tok < a.M) a.y[(int64_t)tok * a.N + row0 + row] = MT::out(acc[nb][q]);
         }
+    }
+    return;
   }
-  __syncthreads();
-  for (int e = threadIdx.x; e < TOK * ROWS; e += blockDim.x) {
-    float s = 0.0f;
-    for (int q = 0; q < NWK; ++q) s += red[(size_t)q * TOK * ROWS + e];
-    part[e] = s;
-  }
-  // every CTA of the cluster has its partial in shared memory
-  cluster.sync();
-  // rank q reduces a slice of the elements over all ranks, in rank order
+  // split-K: element e = tok * ROWS + row belongs to rank e / per; every CTA
+  // stores its partial of e straight into the owner's receive buffer
+  // recv[source rank][e - owner * per] (distributed shared memory), one
+  // cluster barrier publishes all of them, and each owner sums its slice in
+  // rank order.  No remote access follows the barrier.
   const int E = TOK * ROWS;
-  const int per = (E + S - 1) / S;
+  const int per = (E + SK - 1) / SK;
+  if (warp < R) {
+    const int r = lane >> 2, c = lane & 3;
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int row = warp * 16 + r + 8 * (q >> 1);
+        const int tok = nb * 8 + 2 * c + (q & 1);
+        const int e = tok * ROWS + row;
+        const int owner = e / per;
+        cluster.map_shared_rank(part, owner)[rank * per + (e - owner * per)] = acc[nb][q];
+      }
+  }
+  cluster.sync();
+  pdl_wait();  // y may be read by the previous kernel: write only after it completed
   const int e0 = rank * per, e1 = min(E, e0 + per);
   for (int e = e0 + threadIdx.x; e < e1; e += blockDim.x) {
-    float s = 0.0f;
-    for (int q = 0; q < S; ++q) s += cluster.map_shared_rank(part, q)[e];
     const int tok = e / ROWS, row = e % ROWS;
-    if (tok < M) y[(int64_t)tok * N + row0 + row] = MT::out(s);
+    if (tok >= a.M) continue;
+    float sum = 0.0f;
+    for (int q = 0; q < SK; ++q) sum += part[q * per + (e - e0)];
+    a.y[(int64_t)tok * a.N + row0 + row] = MT::out(sum);
   }
-  // keep every CTA's shared memory alive until all remote reads are done
-  cluster.sync();
 }
 
 }  // namespace bq

@@ -3,18 +3,26 @@
 // Method: GreenBitAI article ("只需单卡 RTX 3090 ..."), classic Group-wise MinMax,
 // INT4 / group 128 and INT2 / group 64; arithmetic per
 // "大模型量化实战：从原理到4-bit部署的完整指南" section 2.2 and "低比特量化",
-// section "Zero Point".  See group_params() / code_of() in common.cuh.
+// section "Zero Point".  See group_params() / code_pair() in common.cuh.
 //
 // HBM-bound: 2 bytes read per weight, b/8 + 5/g bytes written.  Two kernels:
 //   * canonical layout: a thread owns 8 consecutive weights (one 16-byte
 //     load), a group spans g/8 adjacent lanes and is reduced with shuffles;
 //     the thread writes its 8 codes as one 32-bit (4-bit) or 16-bit (2-bit)
-//     word.
+//     word; scales / zeros row-major [rows, cols/g].
 //   * interleaved layout: a warp owns a unit of 16 rows x U columns
 //     (U = max(tile width, g)); lane L loads exactly the weights whose codes
-//     form its own 16-byte lane slot of each 512-byte tile, so no permutation
-//     pass is needed; groups are reduced over the 4 lanes sharing a row.
+//     form its own 16-byte slot of each 512-byte tile, so no permutation pass
+//     is needed; groups are reduced over the 4 lanes sharing a row; tiles and
+//     scales / zeros go to their 128-row-block-major places (il_tile_offset,
+//     il_meta_index).  The next unit's weights are loaded before the current
+//     one is computed.
+// The per-element arithmetic runs on packed f32x2 operations (two elements
+// per instruction); the clamp to 2^b - 1 is only evaluated in groups whose
+// largest element needs it.
 #pragma once
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace bq {
@@ -41,22 +49,21 @@ BQ_DEV uint32_t quant8_canonical(uint4 v, bool active, float *s_out, uint8_t *z_
     mn = fmin_nan(mn, __shfl_xor_sync(0xffffffffu, mn, off));
     mx = fmax_nan(mx, __shfl_xor_sync(0xffffffffu, mx, off));
   }
-  GroupParams p = group_params(mn, mx, QMAX);
+  GroupParams p = group_params<QMAX>(mn, mx);
   *s_out = p.s;
   *z_out = (uint8_t)p.z;
   *bad = p.bad;
   uint32_t packed = 0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    packed |= code_of<QMAX, WT == 0>(E::lo(w[i]), p) << (BITS * (2 * i));
-    packed |= code_of<QMAX, WT == 0>(E::hi(w[i]), p) << (BITS * (2 * i + 1));
+    uint2 q = code_pair<QMAX, WT == 0, true>(E::pair(w[i]), p);
+    packed |= (q.x | (q.y << BITS)) << (BITS * 2 * i);
   }
   return packed;
 }
 
 // W viewed flat: element e of the matrix = W[e], groups of G start at
-// multiples of G, codes packed flat.  `base_*` are the block's own arrays
-// (uniform matrix: the whole matrix).
+// multiples of G, codes packed flat.
 template <int WT, int BITS, int G, int UNROLL>
 __global__ void __launch_bounds__(256)
 quantize_canonical_kernel(const uint16_t *__restrict__ W, int64_t elems,
@@ -108,59 +115,89 @@ template <int BITS> struct TileGeom {
   static constexpr int T = (BITS == 4) ? 64 : 128;  // tile width in columns
 };
 
-// Field (bit offset) of the element in row half h (0: row r, 1: row r+8),
-// column pair half hp (0: columns 2c,2c+1; 1: 2c+8,2c+9), odd column `odd`,
-// 16-column run `run` inside its tile.  Returns (word index, bit offset).
+// Bit offset, inside the lane's word, of the even column of slot
+// (h: 0 row r / 1 row r+8, hp: 0 columns 2c,2c+1 / 1 columns 2c+8,2c+9) of
+// 16-column run `run` of the tile; the odd column sits 16 bits higher.
 template <int BITS>
-BQ_DEV constexpr int tile_bit(int run, int h, int hp, int odd) {
-  int slot = h + 2 * hp;
-  if (BITS == 4) return 4 * (slot + 4 * odd);              // word = run
-  return 2 * (4 * (run & 1) + slot + 8 * odd);             // word = run / 2
+BQ_DEV constexpr int tile_bit(int run, int h, int hp) {
+  return BITS == 4 ? 4 * (h + 2 * hp) : 2 * (4 * (run & 1) + h + 2 * hp);
 }
 template <int BITS>
 BQ_DEV constexpr int tile_word(int run) { return BITS == 4 ? run : run / 2; }
 
-// Process one unit: rows row0..row0+15, columns col0..col0+U-1 of a matrix
-// with K columns.  `packed` points to the matrix's packed codes, `scales` /
-// `zeros` to its [rows, K/G] metadata; all indices are relative to them.
-template <int WT, int BITS, int G>
-BQ_DEV bool quantize_unit_tiled(const uint16_t *__restrict__ W, int64_t K, int64_t row0, int64_t col0,
-                                uint8_t *__restrict__ packed, float *__restrict__ scales,
-                                uint8_t *__restrict__ zeros, int lane) {
-  using E = Elem<WT>;
-  constexpr int T = TileGeom<BITS>::T;
-  constexpr int U = (G > T) ? G : T;
-  constexpr int RUNS = U / 16;
-  constexpr int RUNS_PER_G = G / 16;
-  constexpr int NG = U / G;  // groups per row in the unit
-  constexpr int QMAX = (1 << BITS) - 1;
-  const int r = lane >> 2, c = lane & 3;
+template <int BITS, int G> struct UnitGeom {
+  static constexpr int T = TileGeom<BITS>::T;
+  static constexpr int U = (G > T) ? G : T;     // unit width
+  static constexpr int RUNS = U / 16;
+  static constexpr int RUNS_PER_G = G / 16;
+  static constexpr int NG = U / G;              // groups per row in the unit
+  static constexpr int TILES = U / T;
+  static constexpr int RUNS_PER_TILE = T / 16;
+};
 
-  // load: [h][run][hp] half2 pairs
-  uint32_t x[2][RUNS][2];
+// Unit weights of one lane: [h][run][hp] 16-bit pairs.
+template <int BITS, int G> struct UnitRegs {
+  uint32_t x[2][UnitGeom<BITS, G>::RUNS][2];
+};
+
+template <int BITS, int G>
+BQ_DEV void load_unit(UnitRegs<BITS, G> &u, const uint16_t *__restrict__ W, int64_t K, int64_t row0,
+                      int64_t col0, int lane) {
+  const int r = lane >> 2, c = lane & 3;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const uint16_t *rowp = W + (row0 + r + 8 * h) * K + col0 + 2 * c;
 #pragma unroll
-    for (int j = 0; j < RUNS; ++j) {
-      x[h][j][0] = ld_nc_u32(rowp + 16 * j);
-      x[h][j][1] = ld_nc_u32(rowp + 16 * j + 8);
+    for (int j = 0; j < UnitGeom<BITS, G>::RUNS; ++j) {
+      u.x[h][j][0] = ld_nc_u32(rowp + 16 * j);
+      u.x[h][j][1] = ld_nc_u32(rowp + 16 * j + 8);
     }
   }
+}
+
+// Codes of one (row half, group) of the unit ORed into the lane's tile words.
+template <int WT, int BITS, int G, bool CLAMP>
+BQ_DEV void codes_of_group(const UnitRegs<BITS, G> &u, int h, int gi, const GroupParams &p,
+                           uint32_t (&word)[UnitGeom<BITS, G>::TILES][4]) {
+  using UG = UnitGeom<BITS, G>;
+  using E = Elem<WT>;
+  constexpr int QMAX = (1 << BITS) - 1;
+#pragma unroll
+  for (int jj = 0; jj < UG::RUNS_PER_G; ++jj) {
+    const int j = gi * UG::RUNS_PER_G + jj;
+    const int t = j / UG::RUNS_PER_TILE, jt = j % UG::RUNS_PER_TILE;
+#pragma unroll
+    for (int hp = 0; hp < 2; ++hp) {
+      const uint2 q = code_pair<QMAX, WT == 0, CLAMP>(E::pair(u.x[h][j][hp]), p);
+      word[t][tile_word<BITS>(jt)] |= __byte_perm(q.x, q.y, 0x5410) << tile_bit<BITS>(jt, h, hp);
+    }
+  }
+}
+
+// Quantize one loaded unit: rows row0..row0+15, columns col0..col0+U-1 of an
+// N x K matrix; `packed`, `scales`, `zeros` are that matrix's own.
+template <int WT, int BITS, int G>
+BQ_DEV bool quantize_unit(const UnitRegs<BITS, G> &u, int64_t N, int64_t K, int64_t row0, int64_t col0,
+                          uint8_t *__restrict__ packed, float *__restrict__ scales,
+                          uint8_t *__restrict__ zeros, int lane) {
+  using UG = UnitGeom<BITS, G>;
+  using E = Elem<WT>;
+  constexpr int QMAX = (1 << BITS) - 1;
+  const int r = lane >> 2, c = lane & 3;
 
   bool bad_any = false;
-  GroupParams gp[2][NG];
+  GroupParams gp[2][UG::NG];
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
 #pragma unroll
-    for (int gi = 0; gi < NG; ++gi) {
-      uint32_t mn2 = x[h][gi * RUNS_PER_G][0], mx2 = mn2;
+    for (int gi = 0; gi < UG::NG; ++gi) {
+      uint32_t mn2 = u.x[h][gi * UG::RUNS_PER_G][0], mx2 = mn2;
 #pragma unroll
-      for (int j = gi * RUNS_PER_G; j < (gi + 1) * RUNS_PER_G; ++j) {
+      for (int j = gi * UG::RUNS_PER_G; j < (gi + 1) * UG::RUNS_PER_G; ++j) {
 #pragma unroll
         for (int hp = 0; hp < 2; ++hp) {
-          mn2 = E::min2(mn2, x[h][j][hp]);
-          mx2 = E::max2(mx2, x[h][j][hp]);
+          mn2 = E::min2(mn2, u.x[h][j][hp]);
+          mx2 = E::max2(mx2, u.x[h][j][hp]);
         }
       }
       float mn = fmin_nan(E::lo(mn2), E::hi(mn2));
@@ -169,35 +206,27 @@ BQ_DEV bool quantize_unit_tiled(const uint16_t *__restrict__ W, int64_t K, int64
       mx = fmax_nan(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
       mn = fmin_nan(mn, __shfl_xor_sync(0xffffffffu, mn, 2));
       mx = fmax_nan(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      gp[h][gi] = group_params(mn, mx, QMAX);
+      gp[h][gi] = group_params<QMAX>(mn, mx);
       bad_any |= gp[h][gi].bad;
     }
   }
 
-  // codes -> lane words, tile by tile
-  constexpr int TILES = U / T;
-  constexpr int RUNS_PER_TILE = T / 16;
+  uint32_t word[UG::TILES][4];
 #pragma unroll
-  for (int t = 0; t < TILES; ++t) {
-    uint32_t word[4] = {0u, 0u, 0u, 0u};
+  for (int t = 0; t < UG::TILES; ++t)
 #pragma unroll
-    for (int jt = 0; jt < RUNS_PER_TILE; ++jt) {
-      const int j = t * RUNS_PER_TILE + jt;
-      const int gi = j / RUNS_PER_G;
+    for (int i = 0; i < 4; ++i) word[t][i] = 0u;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
+  for (int h = 0; h < 2; ++h)
 #pragma unroll
-        for (int hp = 0; hp < 2; ++hp) {
-          uint32_t pair = x[h][j][hp];
-          uint32_t q0 = code_of<QMAX, WT == 0>(E::lo(pair), gp[h][gi]);
-          uint32_t q1 = code_of<QMAX, WT == 0>(E::hi(pair), gp[h][gi]);
-          word[tile_word<BITS>(jt)] |= (q0 << tile_bit<BITS>(jt, h, hp, 0)) |
-                                       (q1 << tile_bit<BITS>(jt, h, hp, 1));
-        }
-      }
+    for (int gi = 0; gi < UG::NG; ++gi) {
+      if (gp[h][gi].clamp) codes_of_group<WT, BITS, G, true>(u, h, gi, gp[h][gi], word);
+      else codes_of_group<WT, BITS, G, false>(u, h, gi, gp[h][gi], word);
     }
-    const int64_t tile = (row0 / 16) * (K / T) + (col0 / T) + t;
-    st_v4(packed + tile * 512 + lane * 16, make_uint4(word[0], word[1], word[2], word[3]));
+#pragma unroll
+  for (int t = 0; t < UG::TILES; ++t) {
+    const int64_t off = il_tile_offset(row0 / 16, col0 / UG::T + t, N, K, BITS);
+    st_v4(packed + off + lane * 16, make_uint4(word[t][0], word[t][1], word[t][2], word[t][3]));
   }
 
   if (c == 0) {
@@ -205,8 +234,8 @@ BQ_DEV bool quantize_unit_tiled(const uint16_t *__restrict__ W, int64_t K, int64
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
 #pragma unroll
-      for (int gi = 0; gi < NG; ++gi) {
-        const int64_t idx = (row0 + r + 8 * h) * GK + col0 / G + gi;
+      for (int gi = 0; gi < UG::NG; ++gi) {
+        const int64_t idx = il_meta_index(row0 + r + 8 * h, col0 / G + gi, N, GK);
         scales[idx] = gp[h][gi].s;
         zeros[idx] = (uint8_t)gp[h][gi].z;
       }
@@ -220,17 +249,34 @@ __global__ void __launch_bounds__(256)
 quantize_tiled_kernel(const uint16_t *__restrict__ W, int64_t N, int64_t K,
                       uint8_t *__restrict__ packed, float *__restrict__ scales,
                       uint8_t *__restrict__ zeros) {
-  constexpr int T = TileGeom<BITS>::T;
-  constexpr int U = (G > T) ? G : T;
+  using UG = UnitGeom<BITS, G>;
   const int lane = threadIdx.x & 31;
   const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  const int64_t ku = K / U;
+  const int64_t ku = K / UG::U;
   const int64_t units = (N / 16) * ku;
   bool bad = false;
-  for (int64_t u = warp; u < units; u += nwarps) {
-    const int64_t rb = u / ku, kb = u - rb * ku;
-    bad |= quantize_unit_tiled<WT, BITS, G>(W, K, rb * 16, kb * U, packed, scales, zeros, lane);
+  UnitRegs<BITS, G> ua, ub;
+  auto at = [&](int64_t u, int64_t *row0, int64_t *col0) {
+    const int64_t rb = u / ku;
+    *row0 = rb * 16;
+    *col0 = (u - rb * ku) * UG::U;
+  };
+  int64_t r0, c0;
+  int64_t u = warp;
+  if (u < units) { at(u, &r0, &c0); load_unit(ua, W, K, r0, c0, lane); }
+  for (; u < units; u += 2 * nwarps) {
+    const int64_t u1 = u + nwarps;
+    int64_t r1, c1;
+    if (u1 < units) { at(u1, &r1, &c1); load_unit(ub, W, K, r1, c1, lane); }
+    at(u, &r0, &c0);
+    bad |= quantize_unit<WT, BITS, G>(ua, N, K, r0, c0, packed, scales, zeros, lane);
+    if (u1 < units) {
+      const int64_t u2 = u1 + nwarps;
+      int64_t r2, c2;
+      if (u2 < units) { at(u2, &r2, &c2); load_unit(ua, W, K, r2, c2, lane); }
+      bad |= quantize_unit<WT, BITS, G>(ub, N, K, r1, c1, packed, scales, zeros, lane);
+    }
   }
   if (bad) bq_flag(BQ_FLAG_NONFINITE);
 }
@@ -280,11 +326,13 @@ quantize_mixed_tiled_kernel(const uint16_t *__restrict__ W, int64_t N, int64_t K
     const int64_t row_in_blk = (rb % 8) * 16;
     const uint16_t *Wb = W + blk * 128 * K;
     if (bits == 4) {
-      bad |= quantize_unit_tiled<WT, 4, 128>(Wb, K, row_in_blk, kb * U, packed + co, scales + go,
-                                             zeros + go, lane);
+      UnitRegs<4, 128> ur;
+      load_unit(ur, Wb, K, row_in_blk, kb * U, lane);
+      bad |= quantize_unit<WT, 4, 128>(ur, 128, K, row_in_blk, kb * U, packed + co, scales + go, zeros + go, lane);
     } else if (bits == 2) {
-      bad |= quantize_unit_tiled<WT, 2, 64>(Wb, K, row_in_blk, kb * U, packed + co, scales + go,
-                                            zeros + go, lane);
+      UnitRegs<2, 64> ur;
+      load_unit(ur, Wb, K, row_in_blk, kb * U, lane);
+      bad |= quantize_unit<WT, 2, 64>(ur, 128, K, row_in_blk, kb * U, packed + co, scales + go, zeros + go, lane);
     } else {
       badmap = true;
     }

@@ -1,0 +1,55 @@
+// selftest.cuh -- exhaustive check of the quantizer's refined division.
+//
+// The quantizer computes round(x / s) from a correctly rounded quotient
+// obtained by refinement (div_refined, common.cuh) instead of the IEEE
+// division.  Scaling x and s by powers of two scales every step exactly as
+// long as nothing over- or underflows, so comparing against __fdiv_rn for
+// every fp32 divisor of one binade and every fp16 numerator covers every
+// (significand, relative exponent) pair the quantizer meets with fp16 or bf16
+// weights (bf16 significands are a subset of fp16 ones).
+#pragma once
+#include "common.cuh"
+
+namespace bq {
+
+template <int REFINE>
+BQ_DEV float div_refine_n(float x, float s, float r) {
+  float q = __fmul_rn(x, r);
+#pragma unroll
+  for (int i = 0; i < REFINE; ++i) {
+    const float e = __fmaf_rn(-s, q, x);
+    q = __fmaf_rn(e, r, q);
+  }
+  return q;
+}
+
+// One thread per divisor bit pattern; every fp16 numerator with |x| < 64.
+template <int REFINE>
+__global__ void check_division_kernel(uint32_t s_begin, uint32_t s_end, unsigned long long *result) {
+  unsigned long long bad = 0, checked = 0;
+  for (uint64_t sb = s_begin + (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; sb < s_end;
+       sb += (uint64_t)gridDim.x * blockDim.x) {
+    const float s = __uint_as_float((uint32_t)sb);
+    const float r = __frcp_rn(s);
+    for (uint32_t hb = 0; hb < 0x5400u; ++hb) {  // |x| < 64, both signs
+#pragma unroll
+      for (int sign = 0; sign < 2; ++sign) {
+        const float x = __half2float(__ushort_as_half((unsigned short)(hb | (sign << 15))));
+        const float ref = __fdiv_rn(x, s);
+        const float got = div_refine_n<REFINE>(x, s, r);
+        // identical bits, except that a zero quotient may come back as +0 for
+        // x = -0 (both round to the same code)
+        if (__float_as_uint(ref) != __float_as_uint(got) && !(ref == 0.0f && got == 0.0f)) {
+          if (bad == 0 && atomicCAS(result + 2, 0ull, (unsigned long long)sb) == 0ull)
+            result[3] = hb | (sign << 15);
+          ++bad;
+        }
+      }
+    }
+    checked += 2 * 0x5400u;
+  }
+  atomicAdd(result + 0, bad);
+  atomicAdd(result + 1, checked);
+}
+
+}  // namespace bq

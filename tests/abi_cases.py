@@ -73,6 +73,10 @@ def test_linear_validation(L):
     assert lin(L, group=16) == bq.BQ_ERR_UNSUPPORTED
     assert lin(L, N=24) == bq.BQ_ERR_SHAPE
     assert lin(L, K=4032) == bq.BQ_ERR_SHAPE
+    assert lin(L, K=4224) == bq.BQ_ERR_SHAPE                # 4-bit needs K % 256
+    assert lin(L, K=4352, bits=2, group=64) == bq.BQ_ERR_SHAPE   # 2-bit needs K % 512
+    assert lin(L, bm=FAKE, N=4096, K=4352) == bq.BQ_ERR_SHAPE    # mixed needs K % 512
+    assert lin(L, sc=FAKE_MIS) == bq.BQ_ERR_ALIGN          # bulk copies need 16-byte metadata
     assert lin(L, bm=FAKE, N=4000) == bq.BQ_ERR_SHAPE      # mixed needs N % 128
     assert lin(L, x=None) == bq.BQ_ERR_NULL
     assert lin(L, pk=None) == bq.BQ_ERR_NULL

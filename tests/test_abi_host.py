@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(L):
     assert names, "no declarations found"
     for n in names:
         assert hasattr(L, n), n
-    assert set(names) == set(bq.EXPORTS)
+    assert set(names) == set(bq.EXPORTS), set(names) ^ set(bq.EXPORTS)
 
 
 def test_sizes(L):

@@ -74,7 +74,7 @@ def test_decode_shapes_bf16(M, bits, group):
 
 @pytest.mark.parametrize("bits,group", [(4, 32), (4, 64), (4, 256), (2, 32), (2, 128), (2, 256)])
 def test_other_groups(bits, group):
-    N, K = 256, 1024
+    N, K = 272, 1024
     W = synth.normal((N, K), 0.02, seed=group, dtype="f16", device=DEV)
     x = synth.activations(5, K, seed=3, device=DEV)
     pk, sc, ze = bq.bq_quantize(W, bits, group, "interleaved")
@@ -82,12 +82,14 @@ def test_other_groups(bits, group):
     check(y, oracle_y(x, W, bits, group), torch.bfloat16)
 
 
-@pytest.mark.parametrize("N,K", [(16, 128), (48, 256), (16, 4096), (32, 14336), (112, 384)])
+@pytest.mark.parametrize("N,K", [(16, 256), (48, 512), (16, 4096), (32, 14336), (112, 1536), (144, 1024),
+                                 (400, 2560)])
 def test_small_and_ragged(N, K):
+    """Shapes with one row tile, partial 128-row blocks, odd block counts."""
     W = synth.normal((N, K), 0.02, seed=N, dtype="f16", device=DEV)
     x = synth.activations(3, K, seed=K, device=DEV)
     for bits, group in ((4, 128), (2, 64)):
-        if K % (128 if bits == 2 else 128):
+        if K % (256 if bits == 4 else 512):
             continue
         pk, sc, ze = bq.bq_quantize(W, bits, group, "interleaved")
         y = bq.bq_linear(x, pk, sc, ze, N, bits, group)
@@ -104,7 +106,7 @@ def test_heavy_tailed_int2_outliers():
 
 
 def test_more_than_16_tokens():
-    N, K = 512, 1024
+    N, K = 528, 1024
     W = synth.normal((N, K), 0.02, seed=41, dtype="f16", device=DEV)
     x = synth.activations(40, K, seed=42, device=DEV)
     pk, sc, ze = bq.bq_quantize(W, 4, 128, "interleaved")
@@ -139,7 +141,7 @@ def test_channel_mix(M):
 def test_layer_mix_is_uniform_map():
     """Layer-mix assigns one width per layer: a constant map must equal the
     uniform call."""
-    N, K = 512, 1024
+    N, K = 512, 2048
     W = synth.normal((N, K), 0.02, seed=71, dtype="f16", device=DEV)
     x = synth.activations(4, K, seed=72, device=DEV)
     for bits, group in ((4, 128), (2, 64)):

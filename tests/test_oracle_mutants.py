@@ -28,6 +28,9 @@ MUTANTS = {
                          "wrow[k] = (double)((int)codes[n * K + k] + (int)zeros[n * G + j])"),
     "linear_scale_transposed": ("* (double)scales[n * G + j];\n        }\n        for (int64_t m",
                                 "* (double)scales[j * N + n];\n        }\n        for (int64_t m"),
+    "meta_row_major": ("return 128 * G * (n / 128) + g * block_rows(n, rows) + n % 128;",
+                       "return 128 * G * (n / 128) + g * 128 + n % 128;"),
+    "tile_order_row_major": ("*byte_off = block_start + (kt * Rb + t) * 512", "*byte_off = block_start + (t * (cols / T) + kt) * 512"),
     "f16_bias": ("mag = ldexpf((float)(1024 + f), e - 25);", "mag = ldexpf((float)(1024 + f), e - 24);"),
     "f16_subnormal": ("mag = ldexpf((float)f, -24);", "mag = ldexpf((float)f, -25);"),
 }
@@ -41,6 +44,7 @@ PINS = [
     (P.test_page_scale_example, {}),
     (P.test_constant_groups, {}),
     (P.test_interleaved_positions_hand_derived, {}),
+    (P.test_meta_positions_hand_derived, {}),
     (P.test_decode_f16_all_patterns, {}),
     (P.test_invariants, {"bits": 4, "g": 32}),
     (P.test_linear_closed_form, {"bits": 4, "g": 128}),

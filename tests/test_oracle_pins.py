@@ -301,20 +301,43 @@ def test_bf16_rounding():
 def test_interleaved_positions_hand_derived():
     with open(os.path.join(GOLD, "interleaved_positions.txt")) as f:
         rows = [l.split() for l in f if l.strip() and not l.startswith("#")]
-    assert len(rows) >= 16
-    for bits, cols, n, k, byte, bit in (map(int, r) for r in rows):
-        assert O.code_position("interleaved", n, k, cols, bits) == (byte, bit), (bits, cols, n, k)
+    assert len(rows) >= 20
+    for bits, nrows, cols, n, k, byte, bit in (map(int, r) for r in rows):
+        assert O.code_position("interleaved", n, k, nrows, cols, bits) == (byte, bit), (bits, nrows, cols, n, k)
+
+
+def test_meta_positions_hand_derived():
+    with open(os.path.join(GOLD, "meta_positions.txt")) as f:
+        rows = [l.split() for l in f if l.strip() and not l.startswith("#")]
+    assert len(rows) >= 11
+    for layout, n, g, nrows, G, idx in rows:
+        assert O.meta_index(layout, int(n), int(g), int(nrows), int(G)) == int(idx), (layout, n, g, nrows, G)
+
+
+@pytest.mark.parametrize("layout", ["canonical", "interleaved"])
+def test_meta_layout_bijection(layout):
+    rows, G = 144, 24
+    seen = {O.meta_index(layout, n, g, rows, G) for n in range(rows) for g in range(G)}
+    assert seen == set(range(rows * G))
+    rng = np.random.default_rng(1)
+    sc = rng.normal(size=(rows, G)).astype(np.float32)
+    ze = rng.integers(0, 16, (rows, G)).astype(np.uint8)
+    ps, pz = O.pack_meta(sc, ze, layout)
+    for n in range(rows):
+        for g in range(G):
+            i = O.meta_index(layout, n, g, rows, G)
+            assert ps[i] == sc[n, g] and pz[i] == ze[n, g]
 
 
 @pytest.mark.parametrize("bits", [2, 4])
 @pytest.mark.parametrize("layout", ["canonical", "interleaved"])
 def test_pack_bijection(bits, layout):
-    N, K = 32, 256
+    N, K = 144, 256
     rng = np.random.default_rng(bits)
     seen = set()
     for n in range(N):
         for k in range(K):
-            seen.add(O.code_position(layout, n, k, K, bits))
+            seen.add(O.code_position(layout, n, k, N, K, bits))
     assert len(seen) == N * K
     assert all(0 <= b < N * K * bits // 8 and o % bits == 0 and o < 8 for b, o in seen)
     codes = rng.integers(0, 1 << bits, (N, K), dtype=np.uint8)

@@ -16,15 +16,17 @@ DEV = "cuda"
 
 
 def oracle_quant(W: torch.Tensor, bits, group, layout, threads=8):
+    """Oracle codes packed in `layout`, scales / zeros in the layout's metadata order."""
     wt = "f16" if W.dtype == torch.float16 else "bf16"
     codes, scales, zeros = O.quantize(synth.bits16(W), wt, bits, group, threads=threads)
-    return O.pack(codes, bits, layout), scales, zeros, codes
+    ms, mz = O.pack_meta(scales, zeros, layout)
+    return O.pack(codes, bits, layout), ms, mz, codes, scales, zeros
 
 
 def gpu_quant(W, bits, group, layout):
     pk, sc, ze = bq.bq_quantize(W, bits, group, layout)
     assert bq.bq_device_status() == bq.BQ_OK
-    return pk.cpu().numpy(), sc.cpu().numpy(), ze.cpu().numpy()
+    return pk.cpu().numpy(), sc.cpu().numpy().reshape(-1), ze.cpu().numpy().reshape(-1)
 
 
 def assert_same(gpu, ref):
@@ -161,13 +163,15 @@ def test_full_size_sampled_blocks(shape, bits, dist):
         W = synth.student_t4(shape, 0.02, seed=8, dtype="f16", device=DEV, outlier_frac=0.001)
     pk, sc, ze = bq.bq_quantize(W, bits, group, "interleaved")
     assert bq.bq_device_status() == bq.BQ_OK
-    blk_bytes = 16 * K * bits // 8
+    # a 128-row block is contiguous in the interleaved layout (codes and metadata)
+    blk_bytes = 128 * K * bits // 8
+    G = K // group
     rng = np.random.default_rng(N + K)
-    for rb in sorted(set([0, N // 16 - 1] + rng.integers(0, N // 16, 6).tolist())):
-        Wb = W[rb * 16:(rb + 1) * 16].contiguous()
-        rpk, rsc, rze, _ = oracle_quant(Wb, bits, group, "interleaved")
-        got = (pk[rb * blk_bytes:(rb + 1) * blk_bytes].cpu().numpy(),
-               sc[rb * 16:(rb + 1) * 16].cpu().numpy(), ze[rb * 16:(rb + 1) * 16].cpu().numpy())
+    for b in sorted(set([0, N // 128 - 1] + rng.integers(0, N // 128, 3).tolist())):
+        Wb = W[b * 128:(b + 1) * 128].contiguous()
+        rpk, rsc, rze = oracle_quant(Wb, bits, group, "interleaved")[:3]
+        got = (pk[b * blk_bytes:(b + 1) * blk_bytes].cpu().numpy(),
+               sc[b * 128 * G:(b + 1) * 128 * G].cpu().numpy(), ze[b * 128 * G:(b + 1) * 128 * G].cpu().numpy())
         assert_same(got, (rpk, rsc, rze))
     del W, pk, sc, ze
     torch.cuda.empty_cache()
@@ -214,7 +218,7 @@ def test_dequantize_f32_bit_exact(layout, bits, group):
     W = synth.normal((64, 1024), 0.02, seed=4, dtype="f16", device=DEV)
     pk, sc, ze = bq.bq_quantize(W, bits, group, layout)
     got = bq.bq_dequantize(pk, sc, ze, 64, 1024, bits, group, layout, torch.float32).cpu().numpy()
-    _, rsc, rze, codes = oracle_quant(W, bits, group, layout)
+    codes, rsc, rze = oracle_quant(W, bits, group, layout)[3:]
     ref = O.dequant_f32(codes, rsc, rze, group)
     assert (got.view(np.uint32) == ref.view(np.uint32)).all()
     # 16-bit outputs: the fp32 value rounded once
