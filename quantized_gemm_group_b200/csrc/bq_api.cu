@@ -9,6 +9,7 @@
 #include "../../include/bq.h"
 #include "common.cuh"
 #include "dequant.cuh"
+#include "gemm.cuh"
 #include "gemv.cuh"
 #include "quantize.cuh"
 #include "selftest.cuh"
@@ -281,6 +282,108 @@ bq_status gemv_dispatch(const uint16_t *x, int M, int64_t K, const uint8_t *pack
   return BQ_ERR_UNSUPPORTED;
 }
 
+// ---------------------------------------------------------------------------
+// prefill GEMM (tcgen05)
+// ---------------------------------------------------------------------------
+
+// Token count from which bq_linear takes the tensor-core GEMM instead of
+// passes of the decode kernel over 16-token blocks.
+constexpr int64_t kGemmMinTokens = 64;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// The driver's tensor-map encoder, looked up once through the runtime (no
+// link-time dependency on libcuda).
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// x [M, K] 16-bit row-major as a 2D tensor map: boxes of 64 columns (128 B,
+// one swizzle atom) x 256 rows, 128-byte swizzle, rows past M read as zero.
+bool make_x_map(CUtensorMap *map, const uint16_t *x, int64_t M, int64_t K, int xt) {
+  EncodeTiledFn enc = encode_tiled();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+  const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)kGemmChunk, (cuuint32_t)kGemmTokTile};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, xt ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                   const_cast<uint16_t *>(x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int XT, int BITS, int G>
+bq_status launch_gemm_t(const uint16_t *x, int64_t M, int64_t K, const GemmArgs &a, cudaStream_t st) {
+  auto kern = gemm_kernel<XT, BITS, G>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GemmSmem::total) != cudaSuccess)
+      return BQ_ERR_CUDA;
+    attr_set = true;
+  }
+  CUtensorMap map;
+  if (!make_x_map(&map, x, M, K, XT)) return BQ_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(a.N / kGemmRowTile), (unsigned)((M + kGemmTokTile - 1) / kGemmTokTile), 1);
+  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)GemmSmem::total;
+  cfg.stream = st;
+  cudaLaunchAttribute attrs[1];
+  int na = 0;
+  if (overlap_mode() >= 1) {
+    attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attrs[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  cfg.attrs = attrs;
+  cfg.numAttrs = na;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, map, a);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return BQ_ERR_CUDA;
+  }
+  return BQ_OK;
+}
+
+// Uniform width, N a multiple of 128 (whole blocks), groups a multiple of 64
+// columns, at least kGemmMinTokens tokens.
+bool gemm_eligible(int64_t M, int64_t N, const uint8_t *bit_map, int group) {
+  return M >= kGemmMinTokens && !bit_map && N % kGemmRowTile == 0 && group % kGemmChunk == 0 &&
+         M <= 65535LL * kGemmTokTile;
+}
+
+template <int XT>
+bq_status gemm_dispatch(const uint16_t *x, int64_t M, int64_t K, const uint8_t *packed, const float *scales,
+                        const uint8_t *zeros, int bits, int group, int64_t N, uint16_t *y, cudaStream_t st) {
+  GemmArgs a = {};
+  a.packed = packed;
+  a.scales = scales;
+  a.zeros = zeros;
+  a.bit_map = nullptr;
+  a.y = y;
+  a.M = M;
+  a.K = K;
+  a.N = N;
+#define BQ_GM(B, G_) \
+  if (bits == B && group == G_) return launch_gemm_t<XT, B, G_>(x, M, K, a, st);
+  BQ_GM(4, 128) BQ_GM(2, 64) BQ_GM(4, 64) BQ_GM(4, 256) BQ_GM(2, 128) BQ_GM(2, 256)
+#undef BQ_GM
+  return BQ_ERR_UNSUPPORTED;
+}
+
 bool linear_group_ok(int bits, int g) {
   (void)bits;
   return g == 32 || g == 64 || g == 128 || g == 256;
@@ -452,7 +555,10 @@ bq_status bq_linear(const void *x, bq_dtype xtype, int64_t M, int64_t K, const v
   const uint16_t *xx = reinterpret_cast<const uint16_t *>(x);
   uint16_t *yy = reinterpret_cast<uint16_t *>(y);
   const uint8_t *pk = reinterpret_cast<const uint8_t *>(packed);
-  // Token blocks of at most 16 go through the decode kernel.
+  if (gemm_eligible(M, N, bit_map, group))
+    return (xtype == BQ_BF16) ? gemm_dispatch<1>(xx, M, K, pk, scales, zeros, bits, group, N, yy, st)
+                              : gemm_dispatch<0>(xx, M, K, pk, scales, zeros, bits, group, N, yy, st);
+  // Otherwise token blocks of at most 16 go through the decode kernel.
   for (int64_t m0 = 0; m0 < M; m0 += 16) {
     const int mb = (int)((M - m0) < 16 ? (M - m0) : 16);
     bq_status s = (xtype == BQ_BF16)

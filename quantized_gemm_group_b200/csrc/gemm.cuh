@@ -1,0 +1,437 @@
+// gemm.cuh -- prefill / training-forward weight-only linear for large M:
+//   y[m, n] = sum_g s[n, g] * sum_{k in g} x[m, k] * (q[n, k] - z[n, g])
+// on the 5th-generation tensor cores (tcgen05.mma, accumulators in tensor
+// memory).  Same contraction as the decode kernel ("A Survey of Low-bit Large
+// Language Models", section 6.2 weight-only: dequantize, then a 16-bit
+// matmul); here it is a real dense contraction with M >= 2048 tokens.
+//
+// Tile: one 128-row block of the interleaved weight layout (MMA M = 128, the
+// A operand) x 256 tokens (MMA N = 256, the B operand), the whole K range in
+// chunks of 64 columns (one 128-byte swizzle atom of bf16).
+// Warp roles (23 warps):
+//   warp 0      x producer: x chunks by TMA (2D tensor map, 128-byte swizzle,
+//               rows past M zero-filled)
+//   warp 1      TMEM allocation; lane 0 issues tcgen05.mma and commits
+//   warps 2-5   dequantize: exact (q - z) bf16 pairs (LOP3 + 0x4300 magic +
+//               bf16x2 subtract) stored into the 128B-swizzled K-major A
+//               layout, then a proxy fence and an mbarrier arrival
+//   warp 6      code producer: the block's packed codes and zeros by bulk
+//               copies (16 KB stages, contiguous in the layout)
+//   warps 7-22  epilogue (4 per TMEM lane quadrant, 64 token columns each):
+//               per quantization group, tcgen05.ld the group's fp32 partial
+//               (one TMEM lane = one weight row, so the group's scale is one
+//               scalar per thread), FMA into register accumulators, release
+//               the buffer; at the end write y (transposed, bf16)
+// Each group accumulates from zero in one of two TMEM buffers (2 x 256 fp32
+// columns = all 512); the exact integer operand keeps bf16 exact, and the
+// fp32 scale is applied outside the tensor core.
+// Every mbarrier wait is bounded; on expiry the kernel records
+// BQ_FLAG_TIMEOUT, stops, waits (bounded) for the asynchronous work it
+// issued, frees its tensor memory and returns.
+#pragma once
+#include <cuda.h>
+
+#include "common.cuh"
+
+namespace bq {
+
+constexpr int kGemmTokTile = 256;      // MMA N
+constexpr int kGemmRowTile = 128;      // MMA M (one interleaved-layout block)
+constexpr int kGemmChunk = 64;         // K columns per chunk (128 B of bf16)
+constexpr int kGemmXStages = 3;        // x chunk ring (32 KB each)
+constexpr int kGemmAStages = 3;        // dequantized A ring (16 KB each)
+constexpr int kGemmWStages = 2;        // packed-code ring (16 KB + zeros)
+constexpr int kGemmEpiWarps = 16;
+constexpr int kGemmWarpProd = 0, kGemmWarpMma = 1, kGemmWarpDeq0 = 2, kGemmWarpCodes = 6, kGemmWarpEpi0 = 7;
+constexpr int kGemmThreads = (kGemmWarpEpi0 + kGemmEpiWarps) * 32;
+
+template <int BITS, int G> struct GemmG {
+  static constexpr int T = (BITS == 4) ? 64 : 128;    // tile width of the layout
+  static constexpr int SC = (BITS == 4) ? 256 : 512;   // columns per 16 KB code stage
+  static constexpr int CPS = SC / kGemmChunk;          // chunks per code stage
+  static constexpr int GPS = SC / G;                   // groups per code stage
+  static constexpr int CPG = G / kGemmChunk;           // chunks per group (>= 1)
+  static_assert(G % kGemmChunk == 0, "group must be a multiple of 64 columns");
+};
+
+// Shared-memory layout (offsets from a 1024-byte aligned base).
+struct GemmSmem {
+  static constexpr int X_BYTES = kGemmTokTile * 128;   // 32 KB
+  static constexpr int A_BYTES = kGemmRowTile * 128;   // 16 KB
+  static constexpr int W_BYTES = 16384;
+  static constexpr int Z_BYTES = 8 * 128;              // zeros of up to 8 groups x 128 rows
+  static constexpr int x_off = 0;
+  static constexpr int a_off = x_off + kGemmXStages * X_BYTES;
+  static constexpr int w_off = a_off + kGemmAStages * A_BYTES;
+  static constexpr int z_off = w_off + kGemmWStages * W_BYTES;
+  static constexpr int bar_off = z_off + kGemmWStages * Z_BYTES;
+  // barriers: x_full/x_empty [XS], a_full/a_empty [AS], w_full/w_empty [WS],
+  // d_full/d_empty [2], done (abort drain), then the TMEM address and the
+  // abort flag
+  static constexpr int nbar = 2 * kGemmXStages + 2 * kGemmAStages + 2 * kGemmWStages + 5;
+  static constexpr int tmem_off = bar_off + nbar * 8;
+  static constexpr int abort_off = tmem_off + 8;
+  static constexpr int total = abort_off + 8 + 1024;   // + alignment slack
+};
+
+struct GemmArgs {
+  const uint8_t *packed;
+  const float *scales;
+  const uint8_t *zeros;
+  const uint8_t *bit_map;
+  uint16_t *y;
+  int64_t M, K, N;
+};
+
+// ---------------------------------------------------------------------------
+// tcgen05 / TMA primitives
+// ---------------------------------------------------------------------------
+
+// Shared-memory matrix descriptor, K-major, 128-byte swizzle: 8-row groups of
+// 128-byte rows are 1024 bytes apart (stride byte offset); the leading byte
+// offset is unused for this layout; version 1; layout type 2 (128B swizzle).
+BQ_DEV uint64_t umma_desc_sw128(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1u << 16;                  // leading byte offset (16 B, unused)
+  d |= (uint64_t)(1024u >> 4) << 32;        // stride byte offset
+  d |= (uint64_t)1u << 46;                  // descriptor version
+  d |= (uint64_t)2u << 61;                  // 128-byte swizzle
+  return d;
+}
+
+// Instruction descriptor for kind::f16: fp32 accumulate (bits 4-5 = 1), A and
+// B both bf16 (bits 7-9, 10-12 = 1; XT == 1) or both fp16 (0; XT == 0), both
+// K-major, N >> 3 at bit 17, M >> 4 at bit 24.
+template <int XT>
+constexpr uint32_t gemm_idesc() {
+  return (1u << 4) | ((uint32_t)XT << 7) | ((uint32_t)XT << 10) | ((uint32_t)(kGemmTokTile >> 3) << 17) |
+         ((uint32_t)(kGemmRowTile >> 4) << 24);
+}
+
+template <int XT>
+BQ_DEV void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(gemm_idesc<XT>()), "r"(accumulate)
+      : "memory");
+}
+// Arrive on `bar` once every tcgen05.mma issued so far by this thread is done.
+BQ_DEV void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+BQ_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+BQ_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+BQ_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// 8 consecutive fp32 columns of this thread's TMEM lane.
+BQ_DEV void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+  uint32_t r[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+BQ_DEV void tma_load_2d(uint32_t dst, const CUtensorMap *map, int c0, int c1, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+
+// Byte offset of bf16 element (row, k) of a 128-byte-swizzled K-major tile
+// (rows of 64 elements; the 16-byte chunk index is XORed with row % 8).
+BQ_DEV uint32_t sw128_offset(int row, int k) {
+  const int chunk = (k >> 3) ^ (row & 7);
+  return (uint32_t)(row * 128 + chunk * 16 + (k & 7) * 2);
+}
+
+// ---------------------------------------------------------------------------
+// roles
+// ---------------------------------------------------------------------------
+
+// x producer (one thread): every 64-column chunk of the token tile.
+BQ_DEV void gemm_produce_x(const GemmArgs &a, const CUtensorMap *xmap, int tok0, uint32_t sbase, uint32_t bars,
+                           volatile int *abort) {
+  const int nchunks = (int)(a.K / kGemmChunk);
+  const uint32_t x_full = bars, x_empty = bars + 8u * kGemmXStages;
+  int xs = 0, xph = 0, ci = 0;
+  for (; ci < nchunks; ++ci) {
+    if (*abort) break;
+    if (ci >= kGemmXStages && !mbar_wait(x_empty + 8u * xs, xph ^ 1)) { *abort = 1; bq_flag(BQ_FLAG_TIMEOUT); break; }
+    const uint32_t full = x_full + 8u * xs;
+    mbar_arrive_expect_tx(full, (uint32_t)GemmSmem::X_BYTES);
+    tma_load_2d(sbase + GemmSmem::x_off + xs * GemmSmem::X_BYTES, xmap, ci * kGemmChunk, tok0, full);
+    if (++xs == kGemmXStages) { xs = 0; xph ^= 1; }
+  }
+  // the last fill of every slot has landed before the CTA may exit (only
+  // waits on the abort path)
+  for (int j = 1; j <= kGemmXStages && j <= ci; ++j) {
+    const int c = ci - j;
+    mbar_wait(x_full + 8u * (c % kGemmXStages), (c / kGemmXStages) & 1, 1u << 20);
+  }
+}
+
+// Code producer (one thread): 16 KB stages of packed codes plus the zeros of
+// the stage's groups.
+template <int BITS, int G>
+BQ_DEV void gemm_produce_codes(const GemmArgs &a, const uint8_t *pk, const uint8_t *ze, uint32_t sbase,
+                               uint32_t bars, volatile int *abort) {
+  using GG = GemmG<BITS, G>;
+  const int nstages = (int)(a.K / GG::SC);
+  const uint32_t w_full = bars + 8u * (2 * kGemmXStages + 2 * kGemmAStages);
+  const uint32_t w_empty = w_full + 8u * kGemmWStages;
+  constexpr uint32_t zb = (uint32_t)(GG::GPS * 128);
+  int ws = 0, wph = 0, si = 0;
+  for (; si < nstages; ++si) {
+    if (*abort) break;
+    if (si >= kGemmWStages && !mbar_wait(w_empty + 8u * ws, wph ^ 1)) { *abort = 1; bq_flag(BQ_FLAG_TIMEOUT); break; }
+    const uint32_t full = w_full + 8u * ws;
+    mbar_arrive_expect_tx(full, 16384u + zb);
+    bulk_g2s(sbase + GemmSmem::w_off + ws * GemmSmem::W_BYTES, pk + (int64_t)si * 16384, 16384u, full);
+    bulk_g2s(sbase + GemmSmem::z_off + ws * GemmSmem::Z_BYTES, ze + (int64_t)si * GG::GPS * 128, zb, full);
+    if (++ws == kGemmWStages) { ws = 0; wph ^= 1; }
+  }
+  for (int j = 1; j <= kGemmWStages && j <= si; ++j) {
+    const int c = si - j;
+    mbar_wait(w_full + 8u * (c % kGemmWStages), (c / kGemmWStages) & 1, 1u << 20);
+  }
+}
+
+// Dequantize warp d (0..3): row tiles 2d, 2d+1 of every chunk.  The operand
+// is (q - z) as an exact 16-bit float of x's type: bf16 128 + q (0x4300 | q)
+// minus 128 + z, or fp16 1024 + q (0x6400 | q) minus 1024 + z.
+template <int XT, int BITS, int G>
+BQ_DEV void gemm_dequant(const GemmArgs &a, int d, int lane, uint32_t sbase, uint32_t bars, volatile int *abort) {
+  using GG = GemmG<BITS, G>;
+  constexpr uint32_t MASK = (BITS == 4) ? 0x000F000Fu : 0x00030003u;
+  const int nchunks = (int)(a.K / kGemmChunk);
+  const uint32_t a_full = bars + 8u * (2 * kGemmXStages), a_empty = a_full + 8u * kGemmAStages;
+  const uint32_t w_full = bars + 8u * (2 * kGemmXStages + 2 * kGemmAStages);
+  const uint32_t w_empty = w_full + 8u * kGemmWStages;
+  const int r = lane >> 2, c = lane & 3;
+  int as = 0, aph = 0, ws = 0, wph = 0;
+  for (int ci = 0; ci < nchunks; ++ci) {
+    const int cin = ci % GG::CPS;  // chunk inside the code stage
+    if (cin == 0 && !mbar_wait(w_full + 8u * ws, wph)) { *abort = 1; bq_flag(BQ_FLAG_TIMEOUT); break; }
+    if (ci >= kGemmAStages && !mbar_wait(a_empty + 8u * as, aph ^ 1)) { *abort = 1; bq_flag(BQ_FLAG_TIMEOUT); break; }
+    if (*abort) break;
+    const uint32_t wst = sbase + GemmSmem::w_off + ws * GemmSmem::W_BYTES;
+    const uint32_t zst = sbase + GemmSmem::z_off + ws * GemmSmem::Z_BYTES;
+    const uint32_t ast = sbase + GemmSmem::a_off + as * GemmSmem::A_BYTES;
+    // column block and word range of this 64-column chunk
+    const int kt = (BITS == 4) ? cin : cin / 2;
+    const int run0 = (BITS == 4) ? 0 : 4 * (cin & 1);
+    const int gin = (cin * kGemmChunk) / G;  // group inside the code stage
+#pragma unroll
+    for (int tt = 0; tt < 2; ++tt) {
+      const int t = 2 * d + tt;
+      uint4 v;
+      asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                   : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                   : "r"(wst + (kt * 8 + t) * 512 + lane * 16));
+      const uint32_t words[4] = {v.x, v.y, v.z, v.w};
+      uint32_t z0, z1;
+      asm volatile("ld.shared.u8 %0, [%1];" : "=r"(z0) : "r"(zst + gin * 128 + t * 16 + r));
+      asm volatile("ld.shared.u8 %0, [%1];" : "=r"(z1) : "r"(zst + gin * 128 + t * 16 + r + 8));
+      constexpr uint32_t MAGIC = XT ? 0x4300u : 0x6400u;
+      const uint32_t zz0 = (MAGIC | z0) * 0x10001u, zz1 = (MAGIC | z1) * 0x10001u;
+#pragma unroll
+      for (int rr = 0; rr < 4; ++rr) {  // 16-column runs of the chunk
+        const int run = run0 + rr;
+        const uint32_t w = words[BITS == 4 ? run : run / 2];
+        const int base = (BITS == 4) ? 0 : 4 * (run & 1);
+#pragma unroll
+        for (int si = 0; si < 4; ++si) {
+          uint32_t p = (w >> (BITS * (base + si))) & MASK;
+          p |= MAGIC * 0x10001u;
+          uint32_t val;
+          if (XT)
+            asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(val) : "r"(p), "r"((si & 1) ? zz1 : zz0));
+          else
+            asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(val) : "r"(p), "r"((si & 1) ? zz1 : zz0));
+          const int row = t * 16 + r + 8 * (si & 1);
+          const int k = rr * 16 + 8 * (si >> 1) + 2 * c;
+          asm volatile("st.shared.b32 [%0], %1;" ::"r"(ast + sw128_offset(row, k)), "r"(val) : "memory");
+        }
+      }
+    }
+    fence_proxy_async_smem();  // generic-proxy stores -> tensor-core reads
+    __syncwarp();
+    if (lane == 0) mbar_arrive(a_full + 8u * as);
+    if (cin == GG::CPS - 1) {
+      if (lane == 0) mbar_arrive(w_empty + 8u * ws);
+      if (++ws == kGemmWStages) { ws = 0; wph ^= 1; }
+    }
+    if (++as == kGemmAStages) { as = 0; aph ^= 1; }
+  }
+}
+
+// MMA issuer (one thread).
+template <int XT, int BITS, int G>
+BQ_DEV void gemm_mma(const GemmArgs &a, uint32_t tmem, uint32_t sbase, uint32_t bars, volatile int *abort) {
+  using GG = GemmG<BITS, G>;
+  const int nchunks = (int)(a.K / kGemmChunk);
+  const uint32_t x_full = bars, x_empty = bars + 8u * kGemmXStages;
+  const uint32_t a_full = bars + 8u * (2 * kGemmXStages), a_empty = a_full + 8u * kGemmAStages;
+  const uint32_t d_full = bars + 8u * (2 * kGemmXStages + 2 * kGemmAStages + 2 * kGemmWStages);
+  const uint32_t d_empty = d_full + 16u;
+  int xs = 0, xph = 0, as = 0, aph = 0;
+  for (int ci = 0; ci < nchunks; ++ci) {
+    const int g = ci / GG::CPG, cig = ci % GG::CPG;
+    const int buf = g & 1;
+    if (cig == 0 && g >= 2) {
+      if (!mbar_wait(d_empty + 8u * buf, ((g >> 1) - 1) & 1)) { *abort = 1; bq_flag(BQ_FLAG_TIMEOUT); break; }
+      tc_fence_after();
+    }
+    if (!mbar_wait(a_full + 8u * as, aph) || !mbar_wait(x_full + 8u * xs, xph)) {
+      *abort = 1;
+      bq_flag(BQ_FLAG_TIMEOUT);
+      break;
+    }
+    if (*abort) break;
+    tc_fence_after();
+    const uint32_t abase = sbase + GemmSmem::a_off + as * GemmSmem::A_BYTES;
+    const uint32_t xbase = sbase + GemmSmem::x_off + xs * GemmSmem::X_BYTES;
+    const uint32_t d_tmem = tmem + (uint32_t)(buf * kGemmTokTile);
+#pragma unroll
+    for (int kk = 0; kk < kGemmChunk / 16; ++kk)
+      umma_f16<XT>(d_tmem, umma_desc_sw128(abase + kk * 32), umma_desc_sw128(xbase + kk * 32),
+                (cig > 0 || kk > 0) ? 1u : 0u);
+    umma_commit(a_empty + 8u * as);
+    umma_commit(x_empty + 8u * xs);
+    if (cig == GG::CPG - 1) umma_commit(d_full + 8u * buf);
+    if (++as == kGemmAStages) { as = 0; aph ^= 1; }
+    if (++xs == kGemmXStages) { xs = 0; xph ^= 1; }
+  }
+}
+
+// Epilogue warp e (0..15): TMEM lanes 32 (warp % 4) .. +31 (weight rows),
+// token columns 64 (e / 4) .. +63.
+template <int XT, int BITS, int G>
+BQ_DEV void gemm_epilogue(const GemmArgs &a, const float *sc, int e, int warp, int lane, uint32_t tmem,
+                          uint32_t bars, volatile int *abort, int64_t row0, int tok0) {
+  const int ngroups = (int)(a.K / G);
+  const uint32_t d_full = bars + 8u * (2 * kGemmXStages + 2 * kGemmAStages + 2 * kGemmWStages);
+  const uint32_t d_empty = d_full + 16u;
+  const int quad = warp & 3;
+  const int rloc = quad * 32 + lane;          // row inside the block = TMEM lane
+  const int col0 = (e >> 2) * 64;             // token columns of this warp
+  float acc[64];
+#pragma unroll
+  for (int i = 0; i < 64; ++i) acc[i] = 0.0f;
+  const uint32_t lane_addr = ((uint32_t)(quad * 32) << 16);
+  float s_next = __ldg(sc + rloc);            // scale of group 0 (block-major metadata)
+  bool ok = true;
+  for (int g = 0; g < ngroups; ++g) {
+    const int buf = g & 1;
+    const float s = s_next;
+    if (g + 1 < ngroups) s_next = __ldg(sc + (int64_t)(g + 1) * 128 + rloc);
+    if (!mbar_wait(d_full + 8u * buf, (g >> 1) & 1)) { *abort = 1; bq_flag(BQ_FLAG_TIMEOUT); ok = false; break; }
+    tc_fence_after();
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc) {
+      float v[8];
+      tmem_ld8(tmem + lane_addr + (uint32_t)(buf * kGemmTokTile + col0 + cc * 8), v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[cc * 8 + i] = __fmaf_rn(s, v[i], acc[cc * 8 + i]);
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(d_empty + 8u * buf);
+  }
+  if (!ok || *abort) return;
+  // y is [M][N], token-major; this thread owns row (row0 + rloc)
+  const int64_t n = row0 + rloc;
+#pragma unroll 8
+  for (int i = 0; i < 64; ++i) {
+    const int64_t tok = tok0 + col0 + i;
+    if (tok < a.M)
+      a.y[tok * a.N + n] = XT ? __bfloat16_as_ushort(__float2bfloat16_rn(acc[i])) : __half_as_ushort(__float2half_rn(acc[i]));
+  }
+}
+
+// grid = (N / 128 weight blocks, ceil(M / 256) token tiles); 736 threads;
+// one CTA per SM (shared memory), all 512 TMEM columns.
+template <int XT, int BITS, int G>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+gemm_kernel(const __grid_constant__ CUtensorMap xmap, const GemmArgs a) {
+  extern __shared__ __align__(1024) unsigned char gsm_raw[];
+  // 1024-byte aligned base for the swizzled tiles
+  const uint32_t raw = smem_u32(gsm_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  unsigned char *smem = gsm_raw + (sbase - raw);
+  const uint32_t bars = sbase + GemmSmem::bar_off;
+  volatile int *abort = reinterpret_cast<volatile int *>(smem + GemmSmem::abort_off);
+  volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + GemmSmem::tmem_off);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t blk = blockIdx.x;
+  const int64_t row0 = blk * kGemmRowTile;
+  const int tok0 = blockIdx.y * kGemmTokTile;
+
+  if (threadIdx.x == 0) {
+    int b = 0;
+    for (int i = 0; i < kGemmXStages; ++i) { mbar_init(bars + 8u * b++, 1); }
+    for (int i = 0; i < kGemmXStages; ++i) { mbar_init(bars + 8u * b++, 1); }
+    for (int i = 0; i < kGemmAStages; ++i) { mbar_init(bars + 8u * b++, 4); }   // 4 dequant warps
+    for (int i = 0; i < kGemmAStages; ++i) { mbar_init(bars + 8u * b++, 1); }   // MMA commit
+    for (int i = 0; i < kGemmWStages; ++i) { mbar_init(bars + 8u * b++, 1); }
+    for (int i = 0; i < kGemmWStages; ++i) { mbar_init(bars + 8u * b++, 4); }   // 4 dequant warps
+    for (int i = 0; i < 2; ++i) { mbar_init(bars + 8u * b++, 1); }              // d_full: MMA commit
+    for (int i = 0; i < 2; ++i) { mbar_init(bars + 8u * b++, kGemmEpiWarps); }  // d_empty: epilogue warps
+    mbar_init(bars + 8u * b++, 1);                                              // done
+    *abort = 0;
+    mbar_fence_init();
+  }
+  if (warp == kGemmWarpMma) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
+                     sbase + GemmSmem::tmem_off)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const uint8_t *pk = a.packed + blk * kGemmRowTile * a.K * BITS / 8;
+  const float *sc = a.scales + blk * kGemmRowTile * (a.K / G);
+  const uint8_t *ze = a.zeros + blk * kGemmRowTile * (a.K / G);
+
+  pdl_wait();
+  if (warp == kGemmWarpProd) {
+    if (lane == 0) gemm_produce_x(a, &xmap, tok0, sbase, bars, abort);
+  } else if (warp == kGemmWarpMma) {
+    if (lane == 0) gemm_mma<XT, BITS, G>(a, tmem, sbase, bars, abort);
+  } else if (warp == kGemmWarpCodes) {
+    if (lane == 0) gemm_produce_codes<BITS, G>(a, pk, ze, sbase, bars, abort);
+  } else if (warp < kGemmWarpCodes) {
+    gemm_dequant<XT, BITS, G>(a, warp - kGemmWarpDeq0, lane, sbase, bars, abort);
+  } else {
+    gemm_epilogue<XT, BITS, G>(a, sc, warp - kGemmWarpEpi0, warp, lane, tmem, bars, abort, row0, tok0);
+  }
+
+  // everything issued by this CTA has finished before the tensor memory goes
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kGemmWarpMma) {
+    if (*abort && lane == 0) {
+      // wait (bounded) for any MMA still in flight: commit to the barrier
+      // kept for this, then wait for its first phase
+      const uint32_t done = bars + 8u * (2 * kGemmXStages + 2 * kGemmAStages + 2 * kGemmWStages + 4);
+      umma_commit(done);
+      mbar_wait(done, 0, 1u << 20);
+    }
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+  }
+}
+
+}  // namespace bq
