@@ -13,8 +13,10 @@ Printed: ONE JSON line (rank 0).  ``value`` = effective weight GB/s of the
 whole job = (packed codes + scales + zeros + x + y bytes of every linear of
 the step, over all ranks) / max-over-ranks step time.  Extra fields report
 per-M numbers, per-shape numbers, the quantizer over the whole ~7B-weight
-stack, the end-to-end host-buffer path, the roofline of the dominant kernel
-(the decode GEMV) and the CPU oracle baseline.
+stack, the prefill GEMM (tcgen05 path, M = 2048 and 8192 tokens against the
+14336x4096, 4096x14336, 49152x8192 and 8192x49152 weights at INT4 and INT2)
+in TFLOP/s, the end-to-end host-buffer path, the roofline of the dominant
+kernel (the decode GEMV) and the CPU oracle baseline.
 
 Multi-GPU (torchrun): every rank runs its own replica of the stack on its own
 GPU with its own inputs (independent batches, no data-path collective);
@@ -353,6 +355,46 @@ def e2e_numbers(stack, Ms, steps, warmup, world):
     return t, h2d, d2h
 
 
+GEMM_SHAPES = ((14336, 4096), (4096, 14336), (49152, 8192), (8192, 49152))
+
+
+def gemm_numbers(Ms, bf16, bf16_sus, reps=10):
+    """Prefill weight-only GEMM (tcgen05 path of bq_linear) at the prefill
+    shapes: bf16 x N(0,1) [M, K] against INT4 g128 / INT2 g64 weights
+    N(0, 0.015).  TFLOP/s = 2 M N K / CUDA-event time per call (median)."""
+    res = {}
+    for (N, K) in GEMM_SHAPES:
+        W = synth.normal((N, K), 0.015, seed=N + K, dtype="f16", device="cuda")
+        for bits, group in ((4, 128), (2, 64)):
+            pk, sc, ze = bq.bq_quantize(W, bits, group, "interleaved")
+            for M in Ms:
+                x = synth.activations(M, K, seed=M, device="cuda")
+                y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+                for _ in range(3):
+                    bq.bq_linear(x, pk, sc, ze, N, bits, group, out=y)
+                torch.cuda.synchronize()
+                ts = []
+                for _ in range(reps):
+                    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    a.record()
+                    bq.bq_linear(x, pk, sc, ze, N, bits, group, out=y)
+                    b.record()
+                    b.synchronize()
+                    ts.append(a.elapsed_time(b) / 1e3)
+                t = statistics.median(ts)
+                tf = 2.0 * M * N * K / t / 1e12
+                res[f"{N}x{K} INT{bits} M{M}"] = {"us": round(t * 1e6, 1), "TFLOPs": round(tf, 1),
+                                                  "frac_of_measured_bf16_burst": round(tf / bf16, 4),
+                                                  "frac_of_measured_bf16_sustained": round(tf / bf16_sus, 4)}
+                del x, y
+            del pk, sc, ze
+        del W
+        torch.cuda.empty_cache()
+    if bq.bq_device_status() != bq.BQ_OK:
+        raise RuntimeError("GEMM reported a device error")
+    return res
+
+
 def run_gpu(args, world, rank, local):
     hbm, bf16, bf16_sus, peak_kind = peaks()
     bits, group = args.bits, (128 if args.bits == 4 else 64)
@@ -406,6 +448,10 @@ def run_gpu(args, world, rank, local):
                 "us_per_launch_avg": round(t_step / launches_per_step * 1e6, 3)}
 
     extra = {"per_M": per_m, "per_shape": shapes, "quantizer_stack": None}
+    if not args.no_gemm:
+        del g
+        extra["prefill_gemm"] = gemm_numbers((2048, 8192) if not args.quick else (2048,), bf16,
+                                             bf16_sus or bf16)
     if stack.quant:
         qz = stack.quant
         extra["quantizer_stack"] = {"weights": qz["weights"], "ms": round(qz["seconds"] * 1e3, 3),
@@ -504,6 +550,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-quant", action="store_true")
     ap.add_argument("--quick", action="store_true", help="skip the per-shape breakdown")
+    ap.add_argument("--no-gemm", action="store_true", help="skip the prefill GEMM numbers")
     ap.add_argument("--overlap", type=int, default=2, choices=[0, 1, 2],
                     help="bq_linear launch overlap: 0 plain, 1 programmatic dependent launch, "
                          "2 PDL + weight streaming before the wait (weights are static here)")

@@ -251,6 +251,17 @@ BQ_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Non-blocking test of the phase with the given parity.
+BQ_DEV bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 // Bounded wait on the phase with the given parity: false after `limit` polls.
 constexpr uint32_t kWaitLimit = 1u << 22;
 BQ_DEV bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t limit = kWaitLimit) {

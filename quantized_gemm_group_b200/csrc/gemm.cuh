@@ -8,16 +8,15 @@
 // Tile: one 128-row block of the interleaved weight layout (MMA M = 128, the
 // A operand) x 256 tokens (MMA N = 256, the B operand), the whole K range in
 // chunks of 64 columns (one 128-byte swizzle atom of bf16).
-// Warp roles (23 warps):
-//   warp 0      x producer: x chunks by TMA (2D tensor map, 128-byte swizzle,
-//               rows past M zero-filled)
+// Warp roles (22 warps):
+//   warp 0      producer: x chunks by TMA (2D tensor map, 128-byte swizzle,
+//               rows past M zero-filled) and the block's packed codes and
+//               zeros by bulk copies (16 KB stages, contiguous in the layout)
 //   warp 1      TMEM allocation; lane 0 issues tcgen05.mma and commits
 //   warps 2-5   dequantize: exact (q - z) bf16 pairs (LOP3 + 0x4300 magic +
 //               bf16x2 subtract) stored into the 128B-swizzled K-major A
 //               layout, then a proxy fence and an mbarrier arrival
-//   warp 6      code producer: the block's packed codes and zeros by bulk
-//               copies (16 KB stages, contiguous in the layout)
-//   warps 7-22  epilogue (4 per TMEM lane quadrant, 64 token columns each):
+//   warps 6-21  epilogue (4 per TMEM lane quadrant, 64 token columns each):
 //               per quantization group, tcgen05.ld the group's fp32 partial
 //               (one TMEM lane = one weight row, so the group's scale is one
 //               scalar per thread), FMA into register accumulators, release
@@ -25,6 +24,19 @@
 // Each group accumulates from zero in one of two TMEM buffers (2 x 256 fp32
 // columns = all 512); the exact integer operand keeps bf16 exact, and the
 // fp32 scale is applied outside the tensor core.
+// Synchronisation.  Measured on B200: an mbarrier wait (try_wait, test_wait,
+// relaxed or acquire) executed by the thread that has tcgen05.mma
+// instructions outstanding stalls it for ~500 cycles behind them, while a
+// plain shared-memory load does not.  So the MMA thread never waits on an
+// mbarrier: the dequant warps wait for the x bytes of a stage (TMA mbarrier),
+// write the A tile, and publish "chunk c is ready" in a per-warp progress
+// word; the epilogue warps count their releases of each TMEM buffer in a
+// per-buffer counter (a buffer's next use waits for all 16 releases of its
+// previous one, so the counts are exact);
+// the MMA thread polls those words with plain loads, then orders its MMAs
+// after them with tcgen05.fence::after_thread_sync.  It releases stages and
+// announces finished groups with tcgen05.commit onto mbarriers, which the
+// other roles wait on.
 // Every mbarrier wait is bounded; on expiry the kernel records
 // BQ_FLAG_TIMEOUT, stops, waits (bounded) for the asynchronous work it
 // issued, frees its tensor memory and returns.
@@ -39,10 +51,10 @@ constexpr int kGemmTokTile = 256;      // MMA N
 constexpr int kGemmRowTile = 128;      // MMA M (one interleaved-layout block)
 constexpr int kGemmChunk = 64;         // K columns per chunk (128 B of bf16)
 constexpr int kGemmXStages = 3;        // x chunk ring (32 KB each)
-constexpr int kGemmAStages = 3;        // dequantized A ring (16 KB each)
+constexpr int kGemmAStages = 5;        // dequantized A tile ring (16 KB each)
 constexpr int kGemmWStages = 2;        // packed-code ring (16 KB + zeros)
 constexpr int kGemmEpiWarps = 16;
-constexpr int kGemmWarpProd = 0, kGemmWarpMma = 1, kGemmWarpDeq0 = 2, kGemmWarpCodes = 6, kGemmWarpEpi0 = 7;
+constexpr int kGemmWarpProd = 0, kGemmWarpMma = 1, kGemmWarpDeq0 = 2, kGemmWarpEpi0 = 6;
 constexpr int kGemmThreads = (kGemmWarpEpi0 + kGemmEpiWarps) * 32;
 
 template <int BITS, int G> struct GemmG {
@@ -65,11 +77,12 @@ struct GemmSmem {
   static constexpr int w_off = a_off + kGemmAStages * A_BYTES;
   static constexpr int z_off = w_off + kGemmWStages * W_BYTES;
   static constexpr int bar_off = z_off + kGemmWStages * Z_BYTES;
-  // barriers: x_full/x_empty [XS], a_full/a_empty [AS], w_full/w_empty [WS],
-  // d_full/d_empty [2], done (abort drain), then the TMEM address and the
-  // abort flag
-  static constexpr int nbar = 2 * kGemmXStages + 2 * kGemmAStages + 2 * kGemmWStages + 5;
-  static constexpr int tmem_off = bar_off + nbar * 8;
+  // barriers (GemmBars), then the TMEM address and the abort flag
+  static constexpr int nbar = 2 * kGemmXStages + kGemmAStages + 2 * kGemmWStages + 3;
+  static constexpr int prog_off = (bar_off + nbar * 8 + 15) & ~15;  // 4 dequant progress words (16 B)
+  static constexpr int xprog_off = prog_off + 16;                    // x chunks landed
+  static constexpr int epi_off = xprog_off + 4;                      // releases of TMEM buffer 0, 1
+  static constexpr int tmem_off = epi_off + 8 + 4;
   static constexpr int abort_off = tmem_off + 8;
   static constexpr int total = abort_off + 8 + 1024;   // + alignment slack
 };
@@ -82,6 +95,41 @@ struct GemmArgs {
   uint16_t *y;
   int64_t M, K, N;
 };
+
+// Shared-memory addresses of the mbarriers.
+struct GemmBars {
+  uint32_t full, empty;      // [kGemmXStages]: x TMA bytes / one MMA commit
+  uint32_t a_empty;          // [kGemmAStages]: one MMA commit
+  uint32_t w_full, w_empty;  // [kGemmWStages]: code bytes / 4 dequant warps
+  uint32_t d_full;           // [2]: one MMA commit per group
+  uint32_t done;             // MMA drain on the abort path
+  BQ_DEV explicit GemmBars(uint32_t base) {
+    full = base;
+    empty = full + 8u * kGemmXStages;
+    a_empty = empty + 8u * kGemmXStages;
+    w_full = a_empty + 8u * kGemmAStages;
+    w_empty = w_full + 8u * kGemmWStages;
+    d_full = w_empty + 8u * kGemmWStages;
+    done = d_full + 16u;
+  }
+};
+
+BQ_DEV uint4 lds_volatile_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.volatile.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+BQ_DEV uint32_t lds_volatile(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+BQ_DEV void sts_release(uint32_t addr, uint32_t v) {
+  asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+BQ_DEV void red_release_add(uint32_t addr, uint32_t v) {
+  asm volatile("red.release.cta.shared::cta.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
 
 // ---------------------------------------------------------------------------
 // tcgen05 / TMA primitives
@@ -156,51 +204,67 @@ BQ_DEV uint32_t sw128_offset(int row, int k) {
 // roles
 // ---------------------------------------------------------------------------
 
-// x producer (one thread): every 64-column chunk of the token tile.
-BQ_DEV void gemm_produce_x(const GemmArgs &a, const CUtensorMap *xmap, int tok0, uint32_t sbase, uint32_t bars,
-                           volatile int *abort) {
+// Producer (one thread): every 64-column x chunk of the token tile by TMA,
+// and the block's 16 KB code stages plus the zeros of their groups by bulk
+// copies.  It polls both rings without blocking and issues whichever has a
+// free slot; a long stretch without progress counts as a timeout.
+template <int BITS, int G>
+BQ_DEV void gemm_produce(const GemmArgs &a, const CUtensorMap *xmap, const uint8_t *pk, const uint8_t *ze, int tok0,
+                         uint32_t sbase, const GemmBars &B, volatile int *abort) {
+  using GG = GemmG<BITS, G>;
   const int nchunks = (int)(a.K / kGemmChunk);
-  const uint32_t x_full = bars, x_empty = bars + 8u * kGemmXStages;
-  int xs = 0, xph = 0, ci = 0;
-  for (; ci < nchunks; ++ci) {
+  const int nstages = (int)(a.K / GG::SC);
+  constexpr uint32_t zb = (uint32_t)(GG::GPS * 128);
+  const uint32_t xprog = sbase + GemmSmem::xprog_off;
+  int ci = 0, si = 0, xi = 0;  // x chunks issued, code stages issued, x chunks published
+  uint32_t idle = 0;
+  while (xi < nchunks || si < nstages) {
     if (*abort) break;
-    if (ci >= kGemmXStages && !mbar_wait(x_empty + 8u * xs, xph ^ 1)) { *abort = 1; bq_flag(BQ_FLAG_TIMEOUT); break; }
-    const uint32_t full = x_full + 8u * xs;
-    mbar_arrive_expect_tx(full, (uint32_t)GemmSmem::X_BYTES);
-    tma_load_2d(sbase + GemmSmem::x_off + xs * GemmSmem::X_BYTES, xmap, ci * kGemmChunk, tok0, full);
-    if (++xs == kGemmXStages) { xs = 0; xph ^= 1; }
+    bool progress = false;
+    if (si < nstages) {
+      const int ws = si % kGemmWStages;
+      if (si < kGemmWStages || mbar_test_wait(B.w_empty + 8u * ws, ((si / kGemmWStages) & 1) ^ 1)) {
+        const uint32_t full = B.w_full + 8u * ws;
+        mbar_arrive_expect_tx(full, 16384u + zb);
+        bulk_g2s(sbase + GemmSmem::w_off + ws * GemmSmem::W_BYTES, pk + (int64_t)si * 16384, 16384u, full);
+        bulk_g2s(sbase + GemmSmem::z_off + ws * GemmSmem::Z_BYTES, ze + (int64_t)si * GG::GPS * 128, zb, full);
+        ++si;
+        progress = true;
+      }
+    }
+    if (ci < nchunks) {
+      const int st = ci % kGemmXStages;
+      if (ci < kGemmXStages || mbar_test_wait(B.empty + 8u * st, ((ci / kGemmXStages) & 1) ^ 1)) {
+        const uint32_t full = B.full + 8u * st;
+        mbar_arrive_expect_tx(full, (uint32_t)GemmSmem::X_BYTES);
+        tma_load_2d(sbase + GemmSmem::x_off + st * GemmSmem::X_BYTES, xmap, ci * kGemmChunk, tok0, full);
+        ++ci;
+        progress = true;
+      }
+    }
+    // publish the x chunks that have landed, in order
+    if (xi < ci && mbar_test_wait(B.full + 8u * (xi % kGemmXStages), (xi / kGemmXStages) & 1)) {
+      ++xi;
+      sts_release(xprog, (uint32_t)xi);
+      progress = true;
+    }
+    if (progress) {
+      idle = 0;
+    } else if (++idle > (kWaitLimit << 2)) {
+      *abort = 1;
+      bq_flag(BQ_FLAG_TIMEOUT);
+      break;
+    }
   }
   // the last fill of every slot has landed before the CTA may exit (only
-  // waits on the abort path)
+  // waits on the abort path: otherwise the consumers took them all)
   for (int j = 1; j <= kGemmXStages && j <= ci; ++j) {
     const int c = ci - j;
-    mbar_wait(x_full + 8u * (c % kGemmXStages), (c / kGemmXStages) & 1, 1u << 20);
-  }
-}
-
-// Code producer (one thread): 16 KB stages of packed codes plus the zeros of
-// the stage's groups.
-template <int BITS, int G>
-BQ_DEV void gemm_produce_codes(const GemmArgs &a, const uint8_t *pk, const uint8_t *ze, uint32_t sbase,
-                               uint32_t bars, volatile int *abort) {
-  using GG = GemmG<BITS, G>;
-  const int nstages = (int)(a.K / GG::SC);
-  const uint32_t w_full = bars + 8u * (2 * kGemmXStages + 2 * kGemmAStages);
-  const uint32_t w_empty = w_full + 8u * kGemmWStages;
-  constexpr uint32_t zb = (uint32_t)(GG::GPS * 128);
-  int ws = 0, wph = 0, si = 0;
-  for (; si < nstages; ++si) {
-    if (*abort) break;
-    if (si >= kGemmWStages && !mbar_wait(w_empty + 8u * ws, wph ^ 1)) { *abort = 1; bq_flag(BQ_FLAG_TIMEOUT); break; }
-    const uint32_t full = w_full + 8u * ws;
-    mbar_arrive_expect_tx(full, 16384u + zb);
-    bulk_g2s(sbase + GemmSmem::w_off + ws * GemmSmem::W_BYTES, pk + (int64_t)si * 16384, 16384u, full);
-    bulk_g2s(sbase + GemmSmem::z_off + ws * GemmSmem::Z_BYTES, ze + (int64_t)si * GG::GPS * 128, zb, full);
-    if (++ws == kGemmWStages) { ws = 0; wph ^= 1; }
+    mbar_wait(B.full + 8u * (c % kGemmXStages), (c / kGemmXStages) & 1, 1u << 20);
   }
   for (int j = 1; j <= kGemmWStages && j <= si; ++j) {
     const int c = si - j;
-    mbar_wait(w_full + 8u * (c % kGemmWStages), (c / kGemmWStages) & 1, 1u << 20);
+    mbar_wait(B.w_full + 8u * (c % kGemmWStages), (c / kGemmWStages) & 1, 1u << 20);
   }
 }
 
@@ -208,23 +272,27 @@ BQ_DEV void gemm_produce_codes(const GemmArgs &a, const uint8_t *pk, const uint8
 // is (q - z) as an exact 16-bit float of x's type: bf16 128 + q (0x4300 | q)
 // minus 128 + z, or fp16 1024 + q (0x6400 | q) minus 1024 + z.
 template <int XT, int BITS, int G>
-BQ_DEV void gemm_dequant(const GemmArgs &a, int d, int lane, uint32_t sbase, uint32_t bars, volatile int *abort) {
+BQ_DEV void gemm_dequant(const GemmArgs &a, int d, int lane, uint32_t sbase, const GemmBars &B,
+                         volatile int *abort) {
+  const uint32_t prog = sbase + GemmSmem::prog_off + 4u * d;
   using GG = GemmG<BITS, G>;
   constexpr uint32_t MASK = (BITS == 4) ? 0x000F000Fu : 0x00030003u;
+  constexpr uint32_t MAGIC = XT ? 0x4300u : 0x6400u;
   const int nchunks = (int)(a.K / kGemmChunk);
-  const uint32_t a_full = bars + 8u * (2 * kGemmXStages), a_empty = a_full + 8u * kGemmAStages;
-  const uint32_t w_full = bars + 8u * (2 * kGemmXStages + 2 * kGemmAStages);
-  const uint32_t w_empty = w_full + 8u * kGemmWStages;
   const int r = lane >> 2, c = lane & 3;
-  int as = 0, aph = 0, ws = 0, wph = 0;
+  // byte offset, inside an A tile, of (row r of tile 2d, column 2c); the
+  // 16-byte chunk j of a 128-byte swizzled row sits at (j ^ r) * 16
+  const uint32_t rbase = (uint32_t)((2 * d * 16 + r) * 128 + 4 * c);
+  const uint32_t rx = (uint32_t)(r << 4);
+  int st = 0, ph = 0, ws = 0, wph = 0;
   for (int ci = 0; ci < nchunks; ++ci) {
     const int cin = ci % GG::CPS;  // chunk inside the code stage
-    if (cin == 0 && !mbar_wait(w_full + 8u * ws, wph)) { *abort = 1; bq_flag(BQ_FLAG_TIMEOUT); break; }
-    if (ci >= kGemmAStages && !mbar_wait(a_empty + 8u * as, aph ^ 1)) { *abort = 1; bq_flag(BQ_FLAG_TIMEOUT); break; }
+    if (cin == 0 && !mbar_wait(B.w_full + 8u * ws, wph)) { *abort = 1; bq_flag(BQ_FLAG_TIMEOUT); break; }
+    if (ci >= kGemmAStages && !mbar_wait(B.a_empty + 8u * st, ph ^ 1)) { *abort = 1; bq_flag(BQ_FLAG_TIMEOUT); break; }
     if (*abort) break;
     const uint32_t wst = sbase + GemmSmem::w_off + ws * GemmSmem::W_BYTES;
     const uint32_t zst = sbase + GemmSmem::z_off + ws * GemmSmem::Z_BYTES;
-    const uint32_t ast = sbase + GemmSmem::a_off + as * GemmSmem::A_BYTES;
+    const uint32_t ast = sbase + GemmSmem::a_off + st * GemmSmem::A_BYTES;
     // column block and word range of this 64-column chunk
     const int kt = (BITS == 4) ? cin : cin / 2;
     const int run0 = (BITS == 4) ? 0 : 4 * (cin & 1);
@@ -240,7 +308,6 @@ BQ_DEV void gemm_dequant(const GemmArgs &a, int d, int lane, uint32_t sbase, uin
       uint32_t z0, z1;
       asm volatile("ld.shared.u8 %0, [%1];" : "=r"(z0) : "r"(zst + gin * 128 + t * 16 + r));
       asm volatile("ld.shared.u8 %0, [%1];" : "=r"(z1) : "r"(zst + gin * 128 + t * 16 + r + 8));
-      constexpr uint32_t MAGIC = XT ? 0x4300u : 0x6400u;
       const uint32_t zz0 = (MAGIC | z0) * 0x10001u, zz1 = (MAGIC | z1) * 0x10001u;
 #pragma unroll
       for (int rr = 0; rr < 4; ++rr) {  // 16-column runs of the chunk
@@ -249,66 +316,71 @@ BQ_DEV void gemm_dequant(const GemmArgs &a, int d, int lane, uint32_t sbase, uin
         const int base = (BITS == 4) ? 0 : 4 * (run & 1);
 #pragma unroll
         for (int si = 0; si < 4; ++si) {
-          uint32_t p = (w >> (BITS * (base + si))) & MASK;
-          p |= MAGIC * 0x10001u;
+          // slot si: row r (+8 if si odd), columns 2c, 2c+1 (+8 if si >= 2)
+          const uint32_t p = ((w >> (BITS * (base + si))) & MASK) | (MAGIC * 0x10001u);
           uint32_t val;
           if (XT)
             asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(val) : "r"(p), "r"((si & 1) ? zz1 : zz0));
           else
             asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(val) : "r"(p), "r"((si & 1) ? zz1 : zz0));
-          const int row = t * 16 + r + 8 * (si & 1);
-          const int k = rr * 16 + 8 * (si >> 1) + 2 * c;
-          asm volatile("st.shared.b32 [%0], %1;" ::"r"(ast + sw128_offset(row, k)), "r"(val) : "memory");
+          const uint32_t addr = ast + rbase + (((uint32_t)(2 * rr + (si >> 1)) << 4) ^ rx) +
+                                (uint32_t)(tt * 16 * 128 + (si & 1) * 8 * 128);
+          asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(val) : "memory");
         }
       }
     }
     fence_proxy_async_smem();  // generic-proxy stores -> tensor-core reads
     __syncwarp();
-    if (lane == 0) mbar_arrive(a_full + 8u * as);
+    if (lane == 0) sts_release(prog, (uint32_t)(ci + 1));
     if (cin == GG::CPS - 1) {
-      if (lane == 0) mbar_arrive(w_empty + 8u * ws);
+      if (lane == 0) mbar_arrive(B.w_empty + 8u * ws);
       if (++ws == kGemmWStages) { ws = 0; wph ^= 1; }
     }
-    if (++as == kGemmAStages) { as = 0; aph ^= 1; }
+    if (++st == kGemmAStages) { st = 0; ph ^= 1; }
   }
 }
 
-// MMA issuer (one thread).
+// MMA issuer (one thread).  Chunk ci uses stage ci % S and TMEM buffer g & 1
+// of its group g.  Before chunk c it polls (plain shared loads) until every
+// dequant warp has published c as ready and, when c starts a group g >= 2,
+// until the epilogue has released group g - 2's buffer.
 template <int XT, int BITS, int G>
-BQ_DEV void gemm_mma(const GemmArgs &a, uint32_t tmem, uint32_t sbase, uint32_t bars, volatile int *abort) {
+BQ_DEV void gemm_mma(const GemmArgs &a, uint32_t tmem, uint32_t sbase, const GemmBars &B, volatile int *abort) {
   using GG = GemmG<BITS, G>;
   const int nchunks = (int)(a.K / kGemmChunk);
-  const uint32_t x_full = bars, x_empty = bars + 8u * kGemmXStages;
-  const uint32_t a_full = bars + 8u * (2 * kGemmXStages), a_empty = a_full + 8u * kGemmAStages;
-  const uint32_t d_full = bars + 8u * (2 * kGemmXStages + 2 * kGemmAStages + 2 * kGemmWStages);
-  const uint32_t d_empty = d_full + 16u;
-  int xs = 0, xph = 0, as = 0, aph = 0;
+  const uint32_t prog = sbase + GemmSmem::prog_off, xprog = sbase + GemmSmem::xprog_off;
+  const uint32_t epi = sbase + GemmSmem::epi_off;
+  constexpr uint32_t kSpinLimit = kWaitLimit << 4;
   for (int ci = 0; ci < nchunks; ++ci) {
+    const int xs = ci % kGemmXStages, as = ci % kGemmAStages;
     const int g = ci / GG::CPG, cig = ci % GG::CPG;
-    const int buf = g & 1;
-    if (cig == 0 && g >= 2) {
-      if (!mbar_wait(d_empty + 8u * buf, ((g >> 1) - 1) & 1)) { *abort = 1; bq_flag(BQ_FLAG_TIMEOUT); break; }
-      tc_fence_after();
+    // readiness of chunk ci
+    bool ok = true;
+    for (uint32_t spin = 0;; ++spin) {
+      const uint4 p = lds_volatile_v4(prog);
+      const uint32_t need = (uint32_t)ci;
+      bool ready = p.x > need && p.y > need && p.z > need && p.w > need && lds_volatile(xprog) > need;
+      // buffer g & 1 was last used by group g - 2: all its releases counted
+      if (ready && cig == 0 && g >= 2) ready = lds_volatile(epi + 4u * (g & 1)) >= (uint32_t)(kGemmEpiWarps * (g >> 1));
+      if (ready) break;
+      if (spin > kSpinLimit || *abort) { ok = false; break; }
     }
-    if (!mbar_wait(a_full + 8u * as, aph) || !mbar_wait(x_full + 8u * xs, xph)) {
+    if (!ok) {
+      if (!*abort) bq_flag(BQ_FLAG_TIMEOUT);
       *abort = 1;
-      bq_flag(BQ_FLAG_TIMEOUT);
       break;
     }
-    if (*abort) break;
     tc_fence_after();
     const uint32_t abase = sbase + GemmSmem::a_off + as * GemmSmem::A_BYTES;
     const uint32_t xbase = sbase + GemmSmem::x_off + xs * GemmSmem::X_BYTES;
-    const uint32_t d_tmem = tmem + (uint32_t)(buf * kGemmTokTile);
+    const uint32_t d_tmem = tmem + (uint32_t)((g & 1) * kGemmTokTile);
 #pragma unroll
     for (int kk = 0; kk < kGemmChunk / 16; ++kk)
       umma_f16<XT>(d_tmem, umma_desc_sw128(abase + kk * 32), umma_desc_sw128(xbase + kk * 32),
-                (cig > 0 || kk > 0) ? 1u : 0u);
-    umma_commit(a_empty + 8u * as);
-    umma_commit(x_empty + 8u * xs);
-    if (cig == GG::CPG - 1) umma_commit(d_full + 8u * buf);
-    if (++as == kGemmAStages) { as = 0; aph ^= 1; }
-    if (++xs == kGemmXStages) { xs = 0; xph ^= 1; }
+                   (cig > 0 || kk > 0) ? 1u : 0u);
+    umma_commit(B.empty + 8u * xs);
+    umma_commit(B.a_empty + 8u * as);
+    if (cig == GG::CPG - 1) umma_commit(B.d_full + 8u * (g & 1));
   }
 }
 
@@ -316,10 +388,10 @@ BQ_DEV void gemm_mma(const GemmArgs &a, uint32_t tmem, uint32_t sbase, uint32_t 
 // token columns 64 (e / 4) .. +63.
 template <int XT, int BITS, int G>
 BQ_DEV void gemm_epilogue(const GemmArgs &a, const float *sc, int e, int warp, int lane, uint32_t tmem,
-                          uint32_t bars, volatile int *abort, int64_t row0, int tok0) {
+                          uint32_t sbase, const GemmBars &B, volatile int *abort, int64_t row0, int tok0) {
   const int ngroups = (int)(a.K / G);
-  const uint32_t d_full = bars + 8u * (2 * kGemmXStages + 2 * kGemmAStages + 2 * kGemmWStages);
-  const uint32_t d_empty = d_full + 16u;
+  const uint32_t d_full = B.d_full;
+  const uint32_t epi = sbase + GemmSmem::epi_off;
   const int quad = warp & 3;
   const int rloc = quad * 32 + lane;          // row inside the block = TMEM lane
   const int col0 = (e >> 2) * 64;             // token columns of this warp
@@ -344,7 +416,7 @@ BQ_DEV void gemm_epilogue(const GemmArgs &a, const float *sc, int e, int warp, i
     }
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(d_empty + 8u * buf);
+    if (lane == 0) red_release_add(epi + 4u * buf, 1u);  // buffer g & 1 is free again
   }
   if (!ok || *abort) return;
   // y is [M][N], token-major; this thread owns row (row0 + rloc)
@@ -357,7 +429,7 @@ BQ_DEV void gemm_epilogue(const GemmArgs &a, const float *sc, int e, int warp, i
   }
 }
 
-// grid = (N / 128 weight blocks, ceil(M / 256) token tiles); 736 threads;
+// grid = (N / 128 weight blocks, ceil(M / 256) token tiles); 704 threads;
 // one CTA per SM (shared memory), all 512 TMEM columns.
 template <int XT, int BITS, int G>
 __global__ void __launch_bounds__(kGemmThreads, 1)
@@ -367,7 +439,6 @@ gemm_kernel(const __grid_constant__ CUtensorMap xmap, const GemmArgs a) {
   const uint32_t raw = smem_u32(gsm_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
   unsigned char *smem = gsm_raw + (sbase - raw);
-  const uint32_t bars = sbase + GemmSmem::bar_off;
   volatile int *abort = reinterpret_cast<volatile int *>(smem + GemmSmem::abort_off);
   volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + GemmSmem::tmem_off);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -375,17 +446,21 @@ gemm_kernel(const __grid_constant__ CUtensorMap xmap, const GemmArgs a) {
   const int64_t row0 = blk * kGemmRowTile;
   const int tok0 = blockIdx.y * kGemmTokTile;
 
+  const GemmBars B(sbase + GemmSmem::bar_off);
   if (threadIdx.x == 0) {
-    int b = 0;
-    for (int i = 0; i < kGemmXStages; ++i) { mbar_init(bars + 8u * b++, 1); }
-    for (int i = 0; i < kGemmXStages; ++i) { mbar_init(bars + 8u * b++, 1); }
-    for (int i = 0; i < kGemmAStages; ++i) { mbar_init(bars + 8u * b++, 4); }   // 4 dequant warps
-    for (int i = 0; i < kGemmAStages; ++i) { mbar_init(bars + 8u * b++, 1); }   // MMA commit
-    for (int i = 0; i < kGemmWStages; ++i) { mbar_init(bars + 8u * b++, 1); }
-    for (int i = 0; i < kGemmWStages; ++i) { mbar_init(bars + 8u * b++, 4); }   // 4 dequant warps
-    for (int i = 0; i < 2; ++i) { mbar_init(bars + 8u * b++, 1); }              // d_full: MMA commit
-    for (int i = 0; i < 2; ++i) { mbar_init(bars + 8u * b++, kGemmEpiWarps); }  // d_empty: epilogue warps
-    mbar_init(bars + 8u * b++, 1);                                              // done
+    for (int i = 0; i < kGemmXStages; ++i) {
+      mbar_init(B.full + 8u * i, 1);   // the x producer's expect_tx arrival (+ the TMA bytes)
+      mbar_init(B.empty + 8u * i, 1);  // one MMA commit
+    }
+    for (int i = 0; i < kGemmAStages; ++i) mbar_init(B.a_empty + 8u * i, 1);  // one MMA commit
+    for (int i = 0; i < kGemmWStages; ++i) {
+      mbar_init(B.w_full + 8u * i, 1);
+      mbar_init(B.w_empty + 8u * i, 4);   // 4 dequant warps
+    }
+    for (int i = 0; i < 2; ++i) mbar_init(B.d_full + 8u * i, 1);  // one MMA commit per group
+    mbar_init(B.done, 1);
+    volatile uint32_t *words = reinterpret_cast<volatile uint32_t *>(smem + GemmSmem::prog_off);
+    for (int i = 0; i < 7; ++i) words[i] = 0u;  // dequant progress, x landed, released buffers
     *abort = 0;
     mbar_fence_init();
   }
@@ -406,15 +481,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap xmap, const GemmArgs a) {
 
   pdl_wait();
   if (warp == kGemmWarpProd) {
-    if (lane == 0) gemm_produce_x(a, &xmap, tok0, sbase, bars, abort);
+    if (lane == 0) gemm_produce<BITS, G>(a, &xmap, pk, ze, tok0, sbase, B, abort);
   } else if (warp == kGemmWarpMma) {
-    if (lane == 0) gemm_mma<XT, BITS, G>(a, tmem, sbase, bars, abort);
-  } else if (warp == kGemmWarpCodes) {
-    if (lane == 0) gemm_produce_codes<BITS, G>(a, pk, ze, sbase, bars, abort);
-  } else if (warp < kGemmWarpCodes) {
-    gemm_dequant<XT, BITS, G>(a, warp - kGemmWarpDeq0, lane, sbase, bars, abort);
+    if (lane == 0) gemm_mma<XT, BITS, G>(a, tmem, sbase, B, abort);
+  } else if (warp < kGemmWarpEpi0) {
+    gemm_dequant<XT, BITS, G>(a, warp - kGemmWarpDeq0, lane, sbase, B, abort);
   } else {
-    gemm_epilogue<XT, BITS, G>(a, sc, warp - kGemmWarpEpi0, warp, lane, tmem, bars, abort, row0, tok0);
+    gemm_epilogue<XT, BITS, G>(a, sc, warp - kGemmWarpEpi0, warp, lane, tmem, sbase, B, abort, row0, tok0);
   }
 
   // everything issued by this CTA has finished before the tensor memory goes
@@ -424,9 +497,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap xmap, const GemmArgs a) {
     if (*abort && lane == 0) {
       // wait (bounded) for any MMA still in flight: commit to the barrier
       // kept for this, then wait for its first phase
-      const uint32_t done = bars + 8u * (2 * kGemmXStages + 2 * kGemmAStages + 2 * kGemmWStages + 4);
-      umma_commit(done);
-      mbar_wait(done, 0, 1u << 20);
+      umma_commit(B.done);
+      mbar_wait(B.done, 0, 1u << 20);
     }
     __syncwarp();
     tc_fence_after();
