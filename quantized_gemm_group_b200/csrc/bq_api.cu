@@ -332,6 +332,11 @@ bq_status launch_gemm_t(const uint16_t *x, int64_t M, int64_t K, const GemmArgs 
   if (!attr_set) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GemmSmem::total) != cudaSuccess)
       return BQ_ERR_CUDA;
+    // the warpgroups' setmaxnreg shares must fit in the registers the block
+    // is launched with, or the raising warpgroups would wait forever
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return BQ_ERR_CUDA;
+    if ((int64_t)fa.numRegs * kGemmThreads < (int64_t)kGemmRegsNeeded) return BQ_ERR_UNSUPPORTED;
     attr_set = true;
   }
   CUtensorMap map;

@@ -8,15 +8,18 @@
 // Tile: one 128-row block of the interleaved weight layout (MMA M = 128, the
 // A operand) x 256 tokens (MMA N = 256, the B operand), the whole K range in
 // chunks of 64 columns (one 128-byte swizzle atom of bf16).
-// Warp roles (22 warps):
+// Warp roles (24 warps, 6 warpgroups):
 //   warp 0      producer: x chunks by TMA (2D tensor map, 128-byte swizzle,
 //               rows past M zero-filled) and the block's packed codes and
 //               zeros by bulk copies (16 KB stages, contiguous in the layout)
-//   warp 1      TMEM allocation; lane 0 issues tcgen05.mma and commits
-//   warps 2-5   dequantize: exact (q - z) bf16 pairs (LOP3 + 0x4300 magic +
+//   warps 1-2   lane 0 issues tcgen05.mma and commits: warp 1 for the even
+//               groups (TMEM buffer 0), warp 2 for the odd ones; warp 1 also
+//               allocates the tensor memory
+//   warp 3      idle (completes the first warpgroup)
+//   warps 4-7   dequantize: exact (q - z) bf16 pairs (LOP3 + 0x4300 magic +
 //               bf16x2 subtract) stored into the 128B-swizzled K-major A
-//               layout, then a proxy fence and an mbarrier arrival
-//   warps 6-21  epilogue (4 per TMEM lane quadrant, 64 token columns each):
+//               layout, then a proxy fence and a progress word
+//   warps 8-23  epilogue (4 per TMEM lane quadrant, 64 token columns each):
 //               per quantization group, tcgen05.ld the group's fp32 partial
 //               (one TMEM lane = one weight row, so the group's scale is one
 //               scalar per thread), FMA into register accumulators, release
@@ -54,8 +57,15 @@ constexpr int kGemmXStages = 3;        // x chunk ring (32 KB each)
 constexpr int kGemmAStages = 5;        // dequantized A tile ring (16 KB each)
 constexpr int kGemmWStages = 2;        // packed-code ring (16 KB + zeros)
 constexpr int kGemmEpiWarps = 16;
-constexpr int kGemmWarpProd = 0, kGemmWarpMma = 1, kGemmWarpDeq0 = 2, kGemmWarpEpi0 = 6;
-constexpr int kGemmThreads = (kGemmWarpEpi0 + kGemmEpiWarps) * 32;
+constexpr int kGemmWarpProd = 0, kGemmWarpMma = 1, kGemmWarpDeq0 = 4, kGemmWarpEpi0 = 8;
+constexpr int kGemmThreads = (kGemmWarpEpi0 + kGemmEpiWarps) * 32;  // 768
+// Register split (setmaxnreg, per warpgroup of 4 warps): producer / MMA
+// warpgroup, dequant warpgroup, four epilogue warpgroups.  Their sum must
+// not exceed what the block was launched with (threads x registers per
+// thread at launch); the host checks the launch count before the first
+// launch.
+constexpr int kGemmRegsCtl = 56, kGemmRegsDeq = 72, kGemmRegsEpi = 88;
+constexpr int kGemmRegsNeeded = 128 * kGemmRegsCtl + 128 * kGemmRegsDeq + 512 * kGemmRegsEpi;
 
 template <int BITS, int G> struct GemmG {
   static constexpr int T = (BITS == 4) ? 64 : 128;    // tile width of the layout
@@ -78,7 +88,7 @@ struct GemmSmem {
   static constexpr int z_off = w_off + kGemmWStages * W_BYTES;
   static constexpr int bar_off = z_off + kGemmWStages * Z_BYTES;
   // barriers (GemmBars), then the TMEM address and the abort flag
-  static constexpr int nbar = 2 * kGemmXStages + kGemmAStages + 2 * kGemmWStages + 3;
+  static constexpr int nbar = 2 * kGemmXStages + kGemmAStages + 2 * kGemmWStages + 4;
   static constexpr int prog_off = (bar_off + nbar * 8 + 15) & ~15;  // 4 dequant progress words (16 B)
   static constexpr int xprog_off = prog_off + 16;                    // x chunks landed
   static constexpr int epi_off = xprog_off + 4;                      // releases of TMEM buffer 0, 1
@@ -102,7 +112,7 @@ struct GemmBars {
   uint32_t a_empty;          // [kGemmAStages]: one MMA commit
   uint32_t w_full, w_empty;  // [kGemmWStages]: code bytes / 4 dequant warps
   uint32_t d_full;           // [2]: one MMA commit per group
-  uint32_t done;             // MMA drain on the abort path
+  uint32_t done;             // [2]: MMA drain of each issuer on the abort path
   BQ_DEV explicit GemmBars(uint32_t base) {
     full = base;
     empty = full + 8u * kGemmXStages;
@@ -174,16 +184,21 @@ BQ_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;
 BQ_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 BQ_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-// 8 consecutive fp32 columns of this thread's TMEM lane.
-BQ_DEV void tmem_ld8(uint32_t taddr, float (&v)[8]) {
-  uint32_t r[8];
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
-               : "r"(taddr));
+// 16 consecutive fp32 columns of this thread's TMEM lane.
+BQ_DEV void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
+
+template <uint32_t N> BQ_DEV void setmaxnreg_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
+template <uint32_t N> BQ_DEV void setmaxnreg_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
 
 BQ_DEV void tma_load_2d(uint32_t dst, const CUtensorMap *map, int c0, int c1, uint32_t bar) {
   asm volatile(
@@ -340,51 +355,60 @@ BQ_DEV void gemm_dequant(const GemmArgs &a, int d, int lane, uint32_t sbase, con
   }
 }
 
-// MMA issuer (one thread).  Chunk ci uses stage ci % S and TMEM buffer g & 1
-// of its group g.  Before chunk c it polls (plain shared loads) until every
-// dequant warp has published c as ready and, when c starts a group g >= 2,
-// until the epilogue has released group g - 2's buffer.
+// MMA issuers: two threads (lane 0 of warps 1 and 2); issuer `which` owns
+// the groups g with g % 2 == which, i.e. TMEM buffer `which`.  Measured on
+// B200: any shared-memory load (or mbarrier wait) by a thread with
+// tcgen05.mma outstanding returns only after those MMAs have completed, so a
+// single issuer leaves the tensor core idle for ~600 cycles at every
+// readiness check; with two issuers on independent accumulators, one
+// issuer's MMAs run while the other waits.  Before chunk c the issuer polls
+// (plain shared loads) until every dequant warp and the x producer have
+// published c as ready and, when c starts a group g >= 2, until the epilogue
+// has released group g - 2's buffer.
 template <int XT, int BITS, int G>
-BQ_DEV void gemm_mma(const GemmArgs &a, uint32_t tmem, uint32_t sbase, const GemmBars &B, volatile int *abort) {
+BQ_DEV void gemm_mma(const GemmArgs &a, int which, uint32_t tmem, uint32_t sbase, const GemmBars &B,
+                     volatile int *abort) {
   using GG = GemmG<BITS, G>;
-  const int nchunks = (int)(a.K / kGemmChunk);
+  const int ngroups = (int)(a.K / G);
   const uint32_t prog = sbase + GemmSmem::prog_off, xprog = sbase + GemmSmem::xprog_off;
   const uint32_t epi = sbase + GemmSmem::epi_off;
+  const uint32_t d_tmem = tmem + (uint32_t)(which * kGemmTokTile);
   constexpr uint32_t kSpinLimit = kWaitLimit << 4;
-  for (int ci = 0; ci < nchunks; ++ci) {
-    const int xs = ci % kGemmXStages, as = ci % kGemmAStages;
-    const int g = ci / GG::CPG, cig = ci % GG::CPG;
-    // readiness of chunk ci
-    bool ok = true;
-    for (uint32_t spin = 0;; ++spin) {
-      const uint4 p = lds_volatile_v4(prog);
-      const uint32_t need = (uint32_t)ci;
-      bool ready = p.x > need && p.y > need && p.z > need && p.w > need && lds_volatile(xprog) > need;
-      // buffer g & 1 was last used by group g - 2: all its releases counted
-      if (ready && cig == 0 && g >= 2) ready = lds_volatile(epi + 4u * (g & 1)) >= (uint32_t)(kGemmEpiWarps * (g >> 1));
-      if (ready) break;
-      if (spin > kSpinLimit || *abort) { ok = false; break; }
-    }
-    if (!ok) {
-      if (!*abort) bq_flag(BQ_FLAG_TIMEOUT);
-      *abort = 1;
-      break;
-    }
-    tc_fence_after();
-    const uint32_t abase = sbase + GemmSmem::a_off + as * GemmSmem::A_BYTES;
-    const uint32_t xbase = sbase + GemmSmem::x_off + xs * GemmSmem::X_BYTES;
-    const uint32_t d_tmem = tmem + (uint32_t)((g & 1) * kGemmTokTile);
+  for (int g = which; g < ngroups; g += 2) {
+    for (int cig = 0; cig < GG::CPG; ++cig) {
+      const int ci = g * GG::CPG + cig;
+      const int xs = ci % kGemmXStages, as = ci % kGemmAStages;
+      // readiness of chunk ci
+      bool ok = true;
+      for (uint32_t spin = 0;; ++spin) {
+        const uint4 p = lds_volatile_v4(prog);
+        const uint32_t need = (uint32_t)ci;
+        bool ready = p.x > need && p.y > need && p.z > need && p.w > need && lds_volatile(xprog) > need;
+        // buffer `which` was last used by group g - 2: all its releases counted
+        if (ready && cig == 0 && g >= 2) ready = lds_volatile(epi + 4u * which) >= (uint32_t)(kGemmEpiWarps * (g >> 1));
+        if (ready) break;
+        if (spin > kSpinLimit || *abort) { ok = false; break; }
+      }
+      if (!ok) {
+        if (!*abort) bq_flag(BQ_FLAG_TIMEOUT);
+        *abort = 1;
+        return;
+      }
+      tc_fence_after();
+      const uint32_t abase = sbase + GemmSmem::a_off + as * GemmSmem::A_BYTES;
+      const uint32_t xbase = sbase + GemmSmem::x_off + xs * GemmSmem::X_BYTES;
 #pragma unroll
-    for (int kk = 0; kk < kGemmChunk / 16; ++kk)
-      umma_f16<XT>(d_tmem, umma_desc_sw128(abase + kk * 32), umma_desc_sw128(xbase + kk * 32),
-                   (cig > 0 || kk > 0) ? 1u : 0u);
-    umma_commit(B.empty + 8u * xs);
-    umma_commit(B.a_empty + 8u * as);
-    if (cig == GG::CPG - 1) umma_commit(B.d_full + 8u * (g & 1));
+      for (int kk = 0; kk < kGemmChunk / 16; ++kk)
+        umma_f16<XT>(d_tmem, umma_desc_sw128(abase + kk * 32), umma_desc_sw128(xbase + kk * 32),
+                     (cig > 0 || kk > 0) ? 1u : 0u);
+      umma_commit(B.empty + 8u * xs);
+      umma_commit(B.a_empty + 8u * as);
+      if (cig == GG::CPG - 1) umma_commit(B.d_full + 8u * which);
+    }
   }
 }
 
-// Epilogue warp e (0..15): TMEM lanes 32 (warp % 4) .. +31 (weight rows),
+// Epilogue warp e (0..15, warps 8-23): TMEM lanes 32 (warp % 4) .. +31 (weight rows),
 // token columns 64 (e / 4) .. +63.
 template <int XT, int BITS, int G>
 BQ_DEV void gemm_epilogue(const GemmArgs &a, const float *sc, int e, int warp, int lane, uint32_t tmem,
@@ -408,11 +432,11 @@ BQ_DEV void gemm_epilogue(const GemmArgs &a, const float *sc, int e, int warp, i
     if (!mbar_wait(d_full + 8u * buf, (g >> 1) & 1)) { *abort = 1; bq_flag(BQ_FLAG_TIMEOUT); ok = false; break; }
     tc_fence_after();
 #pragma unroll
-    for (int cc = 0; cc < 8; ++cc) {
-      float v[8];
-      tmem_ld8(tmem + lane_addr + (uint32_t)(buf * kGemmTokTile + col0 + cc * 8), v);
+    for (int cc = 0; cc < 4; ++cc) {
+      float v[16];
+      tmem_ld16(tmem + lane_addr + (uint32_t)(buf * kGemmTokTile + col0 + cc * 16), v);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[cc * 8 + i] = __fmaf_rn(s, v[i], acc[cc * 8 + i]);
+      for (int i = 0; i < 16; ++i) acc[cc * 16 + i] = __fmaf_rn(s, v[i], acc[cc * 16 + i]);
     }
     tc_fence_before();
     __syncwarp();
@@ -429,7 +453,7 @@ BQ_DEV void gemm_epilogue(const GemmArgs &a, const float *sc, int e, int warp, i
   }
 }
 
-// grid = (N / 128 weight blocks, ceil(M / 256) token tiles); 704 threads;
+// grid = (N / 128 weight blocks, ceil(M / 256) token tiles); 768 threads;
 // one CTA per SM (shared memory), all 512 TMEM columns.
 template <int XT, int BITS, int G>
 __global__ void __launch_bounds__(kGemmThreads, 1)
@@ -459,6 +483,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap xmap, const GemmArgs a) {
     }
     for (int i = 0; i < 2; ++i) mbar_init(B.d_full + 8u * i, 1);  // one MMA commit per group
     mbar_init(B.done, 1);
+    mbar_init(B.done + 8u, 1);
     volatile uint32_t *words = reinterpret_cast<volatile uint32_t *>(smem + GemmSmem::prog_off);
     for (int i = 0; i < 7; ++i) words[i] = 0u;  // dequant progress, x landed, released buffers
     *abort = 0;
@@ -480,27 +505,31 @@ gemm_kernel(const __grid_constant__ CUtensorMap xmap, const GemmArgs a) {
   const uint8_t *ze = a.zeros + blk * kGemmRowTile * (a.K / G);
 
   pdl_wait();
-  if (warp == kGemmWarpProd) {
-    if (lane == 0) gemm_produce<BITS, G>(a, &xmap, pk, ze, tok0, sbase, B, abort);
-  } else if (warp == kGemmWarpMma) {
-    if (lane == 0) gemm_mma<XT, BITS, G>(a, tmem, sbase, B, abort);
+  if (warp < kGemmWarpDeq0) {
+    setmaxnreg_dec<kGemmRegsCtl>();
+    if (warp == kGemmWarpProd && lane == 0) gemm_produce<BITS, G>(a, &xmap, pk, ze, tok0, sbase, B, abort);
+    if ((warp == kGemmWarpMma || warp == kGemmWarpMma + 1) && lane == 0)
+      gemm_mma<XT, BITS, G>(a, warp - kGemmWarpMma, tmem, sbase, B, abort);
   } else if (warp < kGemmWarpEpi0) {
+    setmaxnreg_dec<kGemmRegsDeq>();
     gemm_dequant<XT, BITS, G>(a, warp - kGemmWarpDeq0, lane, sbase, B, abort);
   } else {
+    setmaxnreg_inc<kGemmRegsEpi>();
     gemm_epilogue<XT, BITS, G>(a, sc, warp - kGemmWarpEpi0, warp, lane, tmem, sbase, B, abort, row0, tok0);
   }
 
   // everything issued by this CTA has finished before the tensor memory goes
   tc_fence_before();
   __syncthreads();
+  if ((warp == kGemmWarpMma || warp == kGemmWarpMma + 1) && *abort && lane == 0) {
+    // wait (bounded) for this issuer's MMAs still in flight: commit to the
+    // barrier kept for this, then wait for its first phase
+    const uint32_t done = B.done + 8u * (warp - kGemmWarpMma);
+    umma_commit(done);
+    mbar_wait(done, 0, 1u << 20);
+  }
+  __syncthreads();
   if (warp == kGemmWarpMma) {
-    if (*abort && lane == 0) {
-      // wait (bounded) for any MMA still in flight: commit to the barrier
-      // kept for this, then wait for its first phase
-      umma_commit(B.done);
-      mbar_wait(B.done, 0, 1u << 20);
-    }
-    __syncwarp();
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
   }
