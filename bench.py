@@ -1,10 +1,12 @@
 #!/usr/bin/env python
 """Benchmark of the W4/W2 weight-only decode path on a Llama-3-8B-shaped stack.
 
-One step = one decode forward through all 32 layers x 7 linears
+One step = one decode forward through all 32 layers x 7 projections
 (q, k, v, o 4096x4096 / 1024x4096; gate, up 14336x4096; down 4096x14336)
-for each batch size M in {1, 4, 16}: 672 bq_linear calls, replayed from one
-CUDA graph.  Weights are synthetic fp16 N(0, 0.02) (seed 1000*layer + module),
+for each batch size M in {1, 4, 16}.  Projections that read the same input
+run as one linear over their weights concatenated along N, as an inference
+engine runs a layer: qkv 6144x4096, o, gate_up 28672x4096, down; 4 bq_linear
+calls per layer, 384 per step, replayed from one CUDA graph.  Weights are synthetic fp16 N(0, 0.02) (seed 1000*layer + module),
 quantized on the GPU by bq_quantize (INT4 group 128 by default); activations
 are bf16 N(0, 1).  The packed stack (3.76 GB at INT4) is far larger than the
 126 MB L2, so every pass streams the weights from HBM; no flush is needed.
@@ -170,6 +172,14 @@ def stack_shapes(layers):
     return [(l, mi, name, N, K) for l in range(layers) for mi, (name, N, K) in enumerate(synth.LLAMA3_8B_LINEARS)]
 
 
+def fused_shapes(layers):
+    """(layer, name, N, K, module indices): the linears of the decode step,
+    q/k/v and gate/up each as one linear over their concatenated weights."""
+    L = synth.LLAMA3_8B_LINEARS
+    return [(l, fname, sum(L[m][1] for m in mods), L[mods[0]][2], mods)
+            for l in range(layers) for fname, mods in synth.LLAMA3_8B_FUSED]
+
+
 # ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
@@ -190,9 +200,27 @@ class Stack:
                 Ws.append(synth.student_t4((N, K), 0.02, seed, "f16", dev, outlier_frac=0.001))
             else:
                 Ws.append(synth.normal((N, K), 0.02, seed, "f16", dev))
-        self.q = []
-        for W, (l, mi, name, N, K) in zip(Ws, self.shapes):
-            self.q.append(bq.bq_quantize(W, bits, group, "interleaved"))
+        # fused linears: one packed / scales / zeros buffer each; every module
+        # is quantized into its slice (the interleaved layout is 128-row-block
+        # major, so stacking whole blocks along N concatenates the buffers)
+        self.fused = fused_shapes(layers)
+        self.fq = []
+        self.q = [None] * len(self.shapes)
+        nlin = len(synth.LLAMA3_8B_LINEARS)
+        for (l, fname, N, K, mods) in self.fused:
+            pk = torch.empty(bq.bq_packed_bytes(N, K, bits), dtype=torch.uint8, device=dev)
+            sc = torch.empty(N * (K // group), dtype=torch.float32, device=dev)
+            ze = torch.empty(N * (K // group), dtype=torch.uint8, device=dev)
+            self.fq.append((pk, sc, ze))
+            r0 = 0
+            for m in mods:
+                Nm = synth.LLAMA3_8B_LINEARS[m][1]
+                cb, gb = bq.bq_packed_bytes(r0, K, bits), r0 * (K // group)
+                ce, ge = bq.bq_packed_bytes(r0 + Nm, K, bits), (r0 + Nm) * (K // group)
+                self.q[l * nlin + m] = (pk[cb:ce], sc[gb:ge], ze[gb:ge])
+                r0 += Nm
+        for W, (l, mi, name, N, K), out in zip(Ws, self.shapes, self.q):
+            bq.bq_quantize(W, bits, group, "interleaved", out=out)
         torch.cuda.synchronize()
         if bq.bq_device_status() != bq.BQ_OK:
             raise RuntimeError("quantizer reported a device error")
@@ -236,19 +264,19 @@ class Stack:
         g = torch.cuda.CUDAGraph()
         with torch.cuda.stream(stream):
             for M in Ms:                                  # warm / lazy init outside capture
-                for i, (l, mi, name, N, K) in enumerate(self.shapes):
-                    pk, sc, ze = self.q[i]
+                for i, (l, fname, N, K, mods) in enumerate(self.fused):
+                    pk, sc, ze = self.fq[i]
                     bq.bq_linear(xs[M][i], pk, sc, ze, N, self.bits, self.group, out=ys[M][i], stream=stream)
             stream.synchronize()
             with torch.cuda.graph(g, stream=stream):
                 for M in Ms:
-                    for i, (l, mi, name, N, K) in enumerate(self.shapes):
-                        pk, sc, ze = self.q[i]
+                    for i, (l, fname, N, K, mods) in enumerate(self.fused):
+                        pk, sc, ze = self.fq[i]
                         bq.bq_linear(xs[M][i], pk, sc, ze, N, self.bits, self.group, out=ys[M][i], stream=stream)
         return g
 
     def step_bytes(self, Ms):
-        return sum(linear_bytes(N, K, self.bits, self.group, M) for M in Ms for (_, _, _, N, K) in self.shapes)
+        return sum(linear_bytes(N, K, self.bits, self.group, M) for M in Ms for (_, _, N, K, _) in self.fused)
 
 
 def time_graph(g, steps, warmup, stream, world, profile=False):
@@ -280,13 +308,12 @@ def per_shape_numbers(stack, M, stream, reps=20):
     """Each distinct shape alone: one graph of 8 rotating weight copies x reps."""
     res = {}
     seen = {}
-    for i, (l, mi, name, N, K) in enumerate(stack.shapes):
-        if name in seen or name in ("k", "up"):          # k == v, up == gate
-            continue
-        seen[name] = i
+    for i, (l, name, N, K, mods) in enumerate(stack.fused):
+        if name not in seen:
+            seen[name] = i
     for name, i in seen.items():
-        (_, _, _, N, K) = stack.shapes[i]
-        idx = [j for j, s in enumerate(stack.shapes) if s[2] == name][:8]
+        (_, _, N, K, _) = stack.fused[i]
+        idx = [j for j, s in enumerate(stack.fused) if s[1] == name][:8]
         x = synth.activations(M, K, seed=5, device="cuda")
         y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
         g = torch.cuda.CUDAGraph()
@@ -294,7 +321,7 @@ def per_shape_numbers(stack, M, stream, reps=20):
             with torch.cuda.graph(g, stream=stream):
                 for _ in range(reps):
                     for j in idx:
-                        pk, sc, ze = stack.q[j]
+                        pk, sc, ze = stack.fq[j]
                         bq.bq_linear(x, pk, sc, ze, N, stack.bits, stack.group, out=y, stream=stream)
         g.replay()
         torch.cuda.synchronize()
@@ -316,8 +343,8 @@ def e2e_numbers(stack, Ms, steps, warmup, world):
     xs_h, ys_h, xs_d, ys_d = {}, {}, {}, {}
     h2d = d2h = 0
     for M in Ms:
-        tot_x = sum(M * K for (_, _, _, N, K) in stack.shapes)
-        tot_y = sum(M * N for (_, _, _, N, K) in stack.shapes)
+        tot_x = sum(M * K for (_, _, N, K, _) in stack.fused)
+        tot_y = sum(M * N for (_, _, N, K, _) in stack.fused)
         xs_h[M] = torch.empty(tot_x, dtype=torch.bfloat16, pin_memory=True)
         xs_h[M].copy_(synth.normal((tot_x,), 1.0, seed=900 + M, dtype="bf16"))
         ys_h[M] = torch.empty(tot_y, dtype=torch.bfloat16, pin_memory=True)
@@ -332,8 +359,8 @@ def e2e_numbers(stack, Ms, steps, warmup, world):
             for M in Ms:
                 xs_d[M].copy_(xs_h[M], non_blocking=True)
                 ox = oy = 0
-                for i, (l, mi, name, N, K) in enumerate(stack.shapes):
-                    pk, sc, ze = stack.q[i]
+                for i, (l, fname, N, K, mods) in enumerate(stack.fused):
+                    pk, sc, ze = stack.fq[i]
                     bq.bq_linear(xs_d[M][ox:ox + M * K].view(M, K), pk, sc, ze, N, stack.bits, stack.group,
                                  out=ys_d[M][oy:oy + M * N].view(M, N), stream=stream)
                     ox += M * K
@@ -405,8 +432,8 @@ def run_gpu(args, world, rank, local):
     bq.bq_set_option(bq.BQ_OPT_LINEAR_OVERLAP, args.overlap)
     Ms = M_SET
     xs = {M: [synth.activations(M, K, seed=10000 * M + i + rank * 7, device="cuda")
-              for i, (_, _, _, N, K) in enumerate(stack.shapes)] for M in Ms}
-    ys = {M: [torch.empty((M, N), dtype=torch.bfloat16, device="cuda") for (_, _, _, N, K) in stack.shapes]
+              for i, (_, _, N, K, _) in enumerate(stack.fused)] for M in Ms}
+    ys = {M: [torch.empty((M, N), dtype=torch.bfloat16, device="cuda") for (_, _, N, K, _) in stack.fused]
           for M in Ms}
     stream = torch.cuda.Stream()
     g = stack.make_graph(Ms, xs, ys, stream)
@@ -432,7 +459,7 @@ def run_gpu(args, world, rank, local):
 
     step_bytes = stack.step_bytes(Ms)
     value = world * step_bytes / t_step / 1e9
-    launches_per_step = len(Ms) * len(stack.shapes)
+    launches_per_step = len(Ms) * len(stack.fused)
 
     # end to end through the C ABI with host buffers
     t_e2e, h2d, d2h = e2e_numbers(stack, Ms, max(1, args.steps // 2), 2, world)
@@ -462,12 +489,13 @@ def run_gpu(args, world, rank, local):
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(t_step * 1e3, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": f"bf16 x int{bits} -> fp32 acc", "data": "synthetic",
-        "config": {"workload": f"Llama-3-8B-shaped decode stack, {args.layers} layers x 7 linears, "
+        "config": {"workload": f"Llama-3-8B-shaped decode stack, {args.layers} layers x 7 projections "
+                               f"(q/k/v and gate/up fused along N: 4 linears per layer), "
                                f"INT{bits} g{group} weight-only, M in {{1,4,16}} per step",
                    "layers": args.layers, "bits": bits, "group": group, "M": list(Ms),
                    "weights": "fp16 N(0,0.02)" if bits == 4 else "fp16 Student-t4 std 0.02 + 0.1% x10 outlier cols",
                    "activations": "bf16 N(0,1)", "l2": "inputs larger than L2 (packed stack %.2f GB)" %
-                   (sum(weight_bytes(N, K, bits, group) for (_, _, _, N, K) in stack.shapes) / 1e9),
+                   (sum(weight_bytes(N, K, bits, group) for (_, _, N, K, _) in stack.fused) / 1e9),
                    "graph": "one CUDA graph per step", "overlap": args.overlap,
                    "parallelism": f"replicas x{world} (independent batches)"},
         "roofline": roofline,
@@ -486,19 +514,23 @@ def run_gpu(args, world, rank, local):
 
 def oracle_sample(threads: int, layers_sample: int = 1, Ms=M_SET, bits=4):
     """Time the CPU oracle's linear layer on a bounded sample of the stack:
-    the first `layers_sample` layers' 7 linears at every M of the step."""
+    the first `layers_sample` layers' linears (q/k/v and gate/up sharing
+    their input) at every M of the step."""
     from oracle import oracle as O  # test infrastructure, CPU baseline only
     group = 128 if bits == 4 else 64
-    shapes = stack_shapes(layers_sample)
     total_bytes = 0
     t_lin = 0.0
-    for (l, mi, name, N, K) in shapes:
-        W = synth.normal((N, K), 0.02, synth.weight_seed(l, mi), "f16", "cpu")
-        codes, scales, zeros = O.quantize(synth.bits16(W), "f16", bits, group, threads=threads)
+    for (l, fname, N, K, mods) in fused_shapes(layers_sample):
+        quant = []
+        for m in mods:
+            Nm = synth.LLAMA3_8B_LINEARS[m][1]
+            W = synth.normal((Nm, K), 0.02, synth.weight_seed(l, m), "f16", "cpu")
+            quant.append(O.quantize(synth.bits16(W), "f16", bits, group, threads=threads))
         for M in Ms:
-            x = O.decode_f64(synth.bits16(synth.activations(M, K, seed=M + mi, device="cpu")), "bf16")
+            x = O.decode_f64(synth.bits16(synth.activations(M, K, seed=M + mods[0], device="cpu")), "bf16")
             t0 = time.perf_counter()
-            O.linear_f64(x, codes, scales, zeros, group, threads=threads)
+            for codes, scales, zeros in quant:
+                O.linear_f64(x, codes, scales, zeros, group, threads=threads)
             t_lin += time.perf_counter() - t0
             total_bytes += linear_bytes(N, K, bits, group, M)
     return total_bytes / t_lin / 1e9, t_lin, total_bytes
@@ -508,7 +540,7 @@ def cpu_baseline(args):
     threads = os.cpu_count() or 1
     gbps, secs, byts = oracle_sample(threads, args.oracle_layers, bits=args.bits)
     return {"value": round(gbps, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
-            "sample": f"first {args.oracle_layers} layer(s) x 7 linears x M in {{1,4,16}} "
+            "sample": f"first {args.oracle_layers} layer(s) x 4 linears (qkv, o, gate_up, down) x M in {{1,4,16}} "
                       f"({byts / 1e6:.1f} MB of weight traffic, {secs:.1f} s); fp64 linear over dequantized weights"}
 
 
@@ -533,7 +565,8 @@ def run_reference(args, world, rank):
         "config": {"workload": f"Llama-3-8B-shaped decode stack, INT{args.bits}, M in {{1,4,16}} "
                                f"(bounded sample: first {args.oracle_layers} layer(s))"},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
-                         "sample": f"first {args.oracle_layers} layer(s) x 7 linears x M in {{1,4,16}} per step"},
+                         "sample": f"first {args.oracle_layers} layer(s) x 4 linears (qkv, o, gate_up, down) "
+                                   f"x M in {{1,4,16}} per step"},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 

@@ -110,6 +110,14 @@ LLAMA3_8B_LINEARS = (
     ("down", 4096, 14336),
 )
 LLAMA3_8B_LAYERS = 32
+# Projections that read the same input, run as one linear over their weights
+# concatenated along N (indices into LLAMA3_8B_LINEARS).
+LLAMA3_8B_FUSED = (
+    ("qkv", (0, 1, 2)),
+    ("o", (3,)),
+    ("gate_up", (4, 5)),
+    ("down", (6,)),
+)
 
 PREFILL_SHAPES = ((14336, 4096), (4096, 14336), (49152, 8192), (8192, 49152))
 

@@ -173,3 +173,25 @@ def test_full_size_sampled_rows(name, N, K, bits):
         rows = np.unique(rows)
         y_ref = oracle_y(x[:M].contiguous(), W, bits, group, rows=torch.from_numpy(rows).to(DEV))
         check(y[:, torch.from_numpy(rows).to(DEV)], y_ref, torch.bfloat16)
+
+
+def test_fused_projections():
+    """q/k/v quantized into consecutive slices of one buffer equal the
+    quantized concatenation, and one linear over it matches the oracle."""
+    K = 2048
+    Ws = [synth.normal((n, K), 0.02, seed=90 + i, dtype="f16", device=DEV) for i, n in enumerate((512, 128, 128))]
+    Wc = torch.cat(Ws)
+    N = Wc.shape[0]
+    pk, sc, ze = bq.bq_quantize(Wc, 4, 128, "interleaved")
+    pk2, sc2, ze2 = torch.empty_like(pk), torch.empty_like(sc), torch.empty_like(ze)
+    r0 = 0
+    for W in Ws:
+        n = W.shape[0]
+        cb, ce = bq.bq_packed_bytes(r0, K, 4), bq.bq_packed_bytes(r0 + n, K, 4)
+        gb, ge = r0 * (K // 128), (r0 + n) * (K // 128)
+        bq.bq_quantize(W, 4, 128, "interleaved", out=(pk2[cb:ce], sc2[gb:ge], ze2[gb:ge]))
+        r0 += n
+    assert torch.equal(pk, pk2) and torch.equal(sc, sc2) and torch.equal(ze, ze2)
+    x = synth.activations(4, K, seed=93, device=DEV)
+    y = bq.bq_linear(x, pk2, sc2, ze2, N, 4, 128)
+    check(y, oracle_y(x, Wc, 4, 128), torch.bfloat16)

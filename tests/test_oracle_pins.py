@@ -421,3 +421,23 @@ def test_mixed_offsets_hand_computed():
     code_off, group_off = O.mixed_offsets([4, 2, 4], 256)
     assert code_off == [0, 16384, 24576, 40960]
     assert group_off == [0, 256, 768, 1024]
+
+
+@pytest.mark.parametrize("bits", [4, 2])
+def test_interleaved_stacks_whole_blocks(bits):
+    """Interleaved layout is 128-row-block major: stacking matrices of whole
+    blocks along N concatenates their packed codes and their metadata, which
+    is what running q/k/v (or gate/up) as one linear relies on."""
+    rng = np.random.default_rng(bits)
+    K = 256 if bits == 4 else 512
+    G = K // (128 if bits == 4 else 64)
+    parts = [rng.integers(0, 1 << bits, size=(n, K), dtype=np.uint8) for n in (256, 128, 128)]
+    whole = np.concatenate(parts)
+    assert (O.pack(whole, bits, "interleaved") ==
+            np.concatenate([O.pack(p, bits, "interleaved") for p in parts])).all()
+    scales = [rng.standard_normal((p.shape[0], G)).astype(np.float32) for p in parts]
+    zeros = [rng.integers(0, 1 << bits, size=(p.shape[0], G), dtype=np.uint8) for p in parts]
+    ms, mz = O.pack_meta(np.concatenate(scales), np.concatenate(zeros), "interleaved")
+    pieces = [O.pack_meta(s, z, "interleaved") for s, z in zip(scales, zeros)]
+    assert (ms.view(np.uint32) == np.concatenate([p[0] for p in pieces]).view(np.uint32)).all()
+    assert (mz == np.concatenate([p[1] for p in pieces])).all()
