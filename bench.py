@@ -51,6 +51,11 @@ MEASURED_PEAKS = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 M_SET = (1, 4, 16)
+# DRAM bytes (read + write) per algorithmic byte of the decode kernel, from
+# the ncu capture of gemv_kernel on gate_up 28672x4096 INT4 at M = 1
+# (profiles/gemv_kernel_gate_up_28672x4096_int4.md: 63.595 MB for 63.37 MB);
+# the kernel reads every weight byte once, so traffic scales with the bytes.
+GEMV_DRAM_PER_ALGO_BYTE = 63.595 / 63.37
 METRIC = "W4/W2 dequant-GEMV weight GB/s (M<=16) & GEMM TFLOP/s (M>=2048) vs roofline"
 
 
@@ -467,7 +472,10 @@ def run_gpu(args, world, rank, local):
 
     achieved = step_bytes / t_step / 1e9   # per-GPU: the GEMV is the only kernel in the step
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                "frac": round(achieved / hbm, 4), "traffic": None,
+                "frac": round(achieved / hbm, 4),
+                "traffic": round(GEMV_DRAM_PER_ALGO_BYTE * step_bytes / launches_per_step) if bits == 4 else None,
+                "traffic_note": "bytes per launch: ncu DRAM bytes per algorithmic byte of the committed capture "
+                                "x this step's algorithmic bytes per launch",
                 "kernel": "gemv_kernel (decode dequant-GEMV, mma.sync bf16)",
                 "peak_kind": peak_kind + " (copy burst)",
                 "frac_of_nominal_8TBps": round(achieved / 8000.0, 4),
