@@ -106,7 +106,7 @@ BQ_DEV uint4 lds_v4(uint32_t addr) {
   return v;
 }
 
-constexpr int kGemvMaxStages = 4;
+constexpr int kGemvMaxStages = 8;
 constexpr int kGemvMaxConsumers = 8;
 
 // Per-width stage geometry: a stage is SC columns of a full 128-row block,
