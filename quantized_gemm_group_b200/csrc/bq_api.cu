@@ -48,6 +48,43 @@ int64_t grid_for(int64_t warps_of_work) {
   return blocks;
 }
 
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// The driver's tensor-map encoder, looked up once through the runtime (no
+// link-time dependency on libcuda).
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// A [rows, cols] 16-bit row-major matrix as a 2D tensor map with boxes of
+// box_cols x box_rows elements, 128-byte swizzle (box_cols * 2 <= 128), rows
+// and columns past the edges read as zero.
+bool make_map_2d(CUtensorMap *map, const void *base, int64_t rows, int64_t cols, bool bf16, int box_cols,
+                 int box_rows) {
+  EncodeTiledFn enc = encode_tiled();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                   const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool valid_bits(int bits) { return bits == 2 || bits == 4; }
 int tile_width(int bits) { return bits == 4 ? 64 : 128; }
 
@@ -71,21 +108,45 @@ bq_status quantize_canonical(const uint16_t *W, int64_t elems, int group, uint8_
   return launch_status();
 }
 
+// Interleaved layout: the TMA-staged kernel, two CTAs per SM, each with a ring
+// of super-units (64 rows x U columns) in about 110 KB of shared memory.
+template <int WT, int BITS, int G>
+bq_status quantize_tma(const uint16_t *W, int64_t N, int64_t K, uint8_t *packed, float *scales, uint8_t *zeros,
+                       cudaStream_t st) {
+  constexpr int U = UnitGeom<BITS, G>::U;
+  constexpr int SU = (U / 64) * 8192;
+  constexpr int kBudget = 113 * 1024;
+  auto kern = quantize_tma_kernel<WT, BITS, G>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kBudget) != cudaSuccess)
+      return BQ_ERR_CUDA;
+    attr_set = true;
+  }
+  int stages = (kBudget - 1024 - 16) / (SU + 16);
+  if (stages > 8) stages = 8;
+  if (stages < 2) return BQ_ERR_UNSUPPORTED;
+  const int smem = stages * SU + 16 * stages + 16 + 1024;
+  CUtensorMap map;
+  if (!make_map_2d(&map, W, N, K, WT == 1, 64, 64)) return BQ_ERR_CUDA;
+  const int64_t nsu = ((N + 63) / 64) * (K / U);
+  int64_t grid = 2 * (int64_t)sm_count();
+  if (grid > nsu) grid = nsu;
+  kern<<<(unsigned)grid, kQtThreads, smem, st>>>(map, N, K, stages, packed, scales, zeros);
+  return launch_status();
+}
+
 template <int WT, int BITS>
 bq_status quantize_tiled(const uint16_t *W, int64_t N, int64_t K, int group, uint8_t *packed, float *scales,
                          uint8_t *zeros, cudaStream_t st) {
-  const int64_t U = group > tile_width(BITS) ? group : tile_width(BITS);
-  const int64_t grid = grid_for((N / 16) * (K / U));
-#define BQ_QT(G)                                                                           \
-  case G:                                                                                  \
-    quantize_tiled_kernel<WT, BITS, G><<<grid, kThreads, 0, st>>>(W, N, K, packed, scales, zeros); \
-    break;
   switch (group) {
-    BQ_QT(16) BQ_QT(32) BQ_QT(64) BQ_QT(128) BQ_QT(256)
+    case 16: return quantize_tma<WT, BITS, 16>(W, N, K, packed, scales, zeros, st);
+    case 32: return quantize_tma<WT, BITS, 32>(W, N, K, packed, scales, zeros, st);
+    case 64: return quantize_tma<WT, BITS, 64>(W, N, K, packed, scales, zeros, st);
+    case 128: return quantize_tma<WT, BITS, 128>(W, N, K, packed, scales, zeros, st);
+    case 256: return quantize_tma<WT, BITS, 256>(W, N, K, packed, scales, zeros, st);
     default: return BQ_ERR_UNSUPPORTED;
   }
-#undef BQ_QT
-  return launch_status();
 }
 
 bool canonical_group_ok(int g) { return g == 8 || g == 16 || g == 32 || g == 64 || g == 128 || g == 256; }
@@ -280,39 +341,10 @@ bq_status gemv_dispatch(const uint16_t *x, int M, int64_t K, const uint8_t *pack
 // passes of the decode kernel over 16-token blocks.
 constexpr int64_t kGemmMinTokens = 64;
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-// The driver's tensor-map encoder, looked up once through the runtime (no
-// link-time dependency on libcuda).
-EncodeTiledFn encode_tiled() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void *p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  });
-  return fn;
-}
-
 // x [M, K] 16-bit row-major as a 2D tensor map: boxes of 64 columns (128 B,
 // one swizzle atom) x 256 rows, 128-byte swizzle, rows past M read as zero.
 bool make_x_map(CUtensorMap *map, const uint16_t *x, int64_t M, int64_t K, int xt) {
-  EncodeTiledFn enc = encode_tiled();
-  if (!enc) return false;
-  const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
-  const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)kGemmChunk, (cuuint32_t)kGemmTokTile};
-  const cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, xt ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
-                   const_cast<uint16_t *>(x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  return make_map_2d(map, x, M, K, xt == 1, 64, kGemmTokTile);
 }
 
 template <int XT, int BITS, int G>

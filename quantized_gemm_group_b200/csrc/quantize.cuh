@@ -282,6 +282,117 @@ quantize_tiled_kernel(const uint16_t *__restrict__ W, int64_t N, int64_t K,
 }
 
 // ---------------------------------------------------------------------------
+// interleaved layout, weights staged by TMA
+// ---------------------------------------------------------------------------
+// The same per-unit arithmetic and stores as quantize_tiled_kernel, with the
+// weights brought into shared memory by TMA instead of held in registers:
+// a super-unit is 64 rows x U columns (four 16-row units), loaded as U / 64
+// boxes of 64 columns x 64 rows with the 128-byte swizzle (16-byte chunk c
+// of row r stored at chunk c ^ (r % 8)), which makes each lane's 4-byte
+// reads conflict-free.  A producer warp keeps a ring of super-units in
+// flight; consumer warps 0-3 take the even ring slots and warps 4-7 the odd
+// ones, warp w quantizing row tile w % 4.  CTAs stride over the super-units.
+constexpr int kQtConsumers = 8;
+constexpr int kQtThreads = 32 * (kQtConsumers + 1);
+
+template <int BITS, int G>
+BQ_DEV void load_unit_smem(UnitRegs<BITS, G> &u, uint32_t su, int t, int lane) {
+  const int r = lane >> 2, c = lane & 3;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int row = 16 * t + r + 8 * h;  // row % 8 == r
+#pragma unroll
+    for (int j = 0; j < UnitGeom<BITS, G>::RUNS; ++j) {
+#pragma unroll
+      for (int hp = 0; hp < 2; ++hp) {
+        const int col = 16 * j + 8 * hp + 2 * c;
+        const uint32_t addr = su + (uint32_t)((col / 64) * 8192 + row * 128 + ((((col % 64) / 8) ^ r) << 4) +
+                                              (col % 8) * 2);
+        asm volatile("ld.shared.b32 %0, [%1];" : "=r"(u.x[h][j][hp]) : "r"(addr));
+      }
+    }
+  }
+}
+
+template <int WT, int BITS, int G>
+__global__ void __launch_bounds__(kQtThreads, 2)
+quantize_tma_kernel(const __grid_constant__ CUtensorMap wmap, int64_t N, int64_t K, int stages,
+                    uint8_t *__restrict__ packed, float *__restrict__ scales, uint8_t *__restrict__ zeros) {
+  using UG = UnitGeom<BITS, G>;
+  constexpr uint32_t SU_BYTES = (uint32_t)(UG::U / 64) * 8192u;
+  extern __shared__ __align__(1024) unsigned char qt_raw[];
+  const uint32_t raw = smem_u32(qt_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;  // the launch adds 1024 bytes of slack
+  const uint32_t bars = sbase + (uint32_t)stages * SU_BYTES;
+  volatile int *abort = reinterpret_cast<volatile int *>(qt_raw + (sbase - raw) + stages * SU_BYTES + 16 * stages);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t ku = K / UG::U;
+  const int64_t nsu = ((N + 63) / 64) * ku;
+  // super-units of this CTA: blockIdx.x, + gridDim.x, ...
+  const int n = (int)((nsu - blockIdx.x + gridDim.x - 1) / gridDim.x);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(bars + 8u * s, 1);
+      mbar_init(bars + 8u * (stages + s), kQtConsumers / 2);
+    }
+    *abort = 0;
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (warp == kQtConsumers) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < n; ++i) {
+        const int slot = i % stages;
+        if (i >= stages && !mbar_wait(bars + 8u * (stages + slot), ((i / stages) & 1) ^ 1)) {
+          *abort = 1;
+          bq_flag(BQ_FLAG_TIMEOUT);
+          break;
+        }
+        const int64_t su = blockIdx.x + (int64_t)i * gridDim.x;
+        const int64_t rb = su / ku;
+        const int col0 = (int)((su - rb * ku) * UG::U), row0 = (int)(rb * 64);
+        const uint32_t full = bars + 8u * slot;
+        mbar_arrive_expect_tx(full, SU_BYTES);
+#pragma unroll
+        for (int b = 0; b < UG::U / 64; ++b)
+          tma_load_2d(sbase + (uint32_t)slot * SU_BYTES + b * 8192u, &wmap, col0 + 64 * b, row0, full);
+        issued = i + 1;
+      }
+      if (*abort) {  // the loads already issued land before the CTA exits
+        for (int i = (issued > stages ? issued - stages : 0); i < issued; ++i)
+          mbar_wait(bars + 8u * (i % stages), (i / stages) & 1, 1u << 20);
+      }
+    }
+    return;
+  }
+  const int par = warp / 4, t = warp % 4;
+  bool bad = false;
+  for (int i = par; i < n; i += 2) {
+    const int slot = i % stages;
+    if (*abort || !mbar_wait(bars + 8u * slot, (i / stages) & 1)) {
+      *abort = 1;
+      bq_flag(BQ_FLAG_TIMEOUT);
+      break;
+    }
+    const int64_t su = blockIdx.x + (int64_t)i * gridDim.x;
+    const int64_t rb = su / ku;
+    const int64_t col0 = (su - rb * ku) * UG::U, row0 = rb * 64 + 16 * t;
+    if (row0 < N) {
+      UnitRegs<BITS, G> u;
+      load_unit_smem<BITS, G>(u, sbase + (uint32_t)slot * SU_BYTES, t, lane);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars + 8u * (stages + slot));
+      bad |= quantize_unit<WT, BITS, G>(u, N, K, row0, col0, packed, scales, zeros, lane);
+    } else {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars + 8u * (stages + slot));
+    }
+  }
+  if (bad) bq_flag(BQ_FLAG_NONFINITE);
+}
+
+// ---------------------------------------------------------------------------
 // mixed precision: per 128-row block width from a device bit map
 // ---------------------------------------------------------------------------
 
