@@ -53,9 +53,9 @@ FALLBACK_BF16_TFLOPS = 1590.0
 M_SET = (1, 4, 16)
 # DRAM bytes (read + write) per algorithmic byte of the decode kernel, from
 # the ncu capture of gemv_kernel on gate_up 28672x4096 INT4 at M = 1
-# (profiles/gemv_kernel_gate_up_28672x4096_int4.md: 63.595 MB for 63.37 MB);
+# (profiles/gemv_kernel_gate_up_28672x4096_int4.md: 63.654 MB for 63.37 MB);
 # the kernel reads every weight byte once, so traffic scales with the bytes.
-GEMV_DRAM_PER_ALGO_BYTE = 63.595 / 63.37
+GEMV_DRAM_PER_ALGO_BYTE = 63.654 / 63.37
 METRIC = "W4/W2 dequant-GEMV weight GB/s (M<=16) & GEMM TFLOP/s (M>=2048) vs roofline"
 
 
@@ -344,7 +344,10 @@ def per_shape_numbers(stack, M, stream, reps=20):
 
 def e2e_numbers(stack, Ms, steps, warmup, world):
     """Same metric through the C ABI with host buffers: every step copies all
-    activations from pinned host memory to the device and all outputs back."""
+    activations from pinned host memory to the device and all outputs back.
+    The copies are pipelined with the compute: the inputs of the next batch
+    size go up while the current one computes, and its outputs come down
+    while the next computes (separate copy streams, events between them)."""
     xs_h, ys_h, xs_d, ys_d = {}, {}, {}, {}
     h2d = d2h = 0
     for M in Ms:
@@ -357,30 +360,50 @@ def e2e_numbers(stack, Ms, steps, warmup, world):
         ys_d[M] = torch.empty(tot_y, dtype=torch.bfloat16, device="cuda")
         h2d += tot_x * 2
         d2h += tot_y * 2
-    stream = torch.cuda.Stream()
+    comp, up, down = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    x_ready = {M: torch.cuda.Event() for M in Ms}     # inputs on the device
+    x_free = {M: torch.cuda.Event() for M in Ms}      # compute done reading them
+    y_ready = {M: torch.cuda.Event() for M in Ms}     # outputs written
+    y_free = {M: torch.cuda.Event() for M in Ms}      # outputs copied down
+    for M in Ms:
+        x_free[M].record(comp)
+        y_free[M].record(down)
 
     def one_step():
-        with torch.cuda.stream(stream):
-            for M in Ms:
+        for M in Ms:
+            with torch.cuda.stream(up):
+                up.wait_event(x_free[M])
                 xs_d[M].copy_(xs_h[M], non_blocking=True)
+                x_ready[M].record(up)
+        for M in Ms:
+            with torch.cuda.stream(comp):
+                comp.wait_event(x_ready[M])
+                comp.wait_event(y_free[M])
                 ox = oy = 0
                 for i, (l, fname, N, K, mods) in enumerate(stack.fused):
                     pk, sc, ze = stack.fq[i]
                     bq.bq_linear(xs_d[M][ox:ox + M * K].view(M, K), pk, sc, ze, N, stack.bits, stack.group,
-                                 out=ys_d[M][oy:oy + M * N].view(M, N), stream=stream)
+                                 out=ys_d[M][oy:oy + M * N].view(M, N), stream=comp)
                     ox += M * K
                     oy += M * N
+                x_free[M].record(comp)
+                y_ready[M].record(comp)
+            with torch.cuda.stream(down):
+                down.wait_event(y_ready[M])
                 ys_h[M].copy_(ys_d[M], non_blocking=True)
+                y_free[M].record(down)
 
     for _ in range(warmup):
         one_step()
-    stream.synchronize()
+    torch.cuda.synchronize()
     barrier(world)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
+    a.record(up)
     for _ in range(steps):
         one_step()
-    b.record(stream)
+    for M in Ms:
+        up.wait_event(y_free[M])       # the last outputs are on the host
+    b.record(up)
     b.synchronize()
     barrier(world)
     t = a.elapsed_time(b) / 1e3 / steps
