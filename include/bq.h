@@ -171,7 +171,8 @@ bq_status bq_dequantize(const void *packed, const float *scales, const uint8_t *
  *   bit_map  NULL for a uniform matrix (bits, group used; production pairs
  *            (4, 128) and (2, 64), tests also group 32 and 256), else a DEVICE
  *            bit map as in bq_quantize_mixed (bits, group ignored)
- *   y        [M, N] of xtype, written in full
+ *   y        [M, N] of xtype, written in full (K == 0: zeros, x not read;
+ *            M == 0 or N == 0: nothing is done)
  * Products are accumulated in fp32 per group on exact (q - z) operands, then
  * scaled by the group's fp32 s and summed in fp32; y is rounded once.
  * M <= 16 runs the decode kernel (split-K dequant-GEMV on tensor cores);

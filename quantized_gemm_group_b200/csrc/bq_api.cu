@@ -571,11 +571,12 @@ bq_status bq_linear(const void *x, bq_dtype xtype, int64_t M, int64_t K, const v
     if (N % 16 || K % (bits == 4 ? 256 : 512)) return BQ_ERR_SHAPE;
   }
   if (M == 0 || N == 0) return BQ_OK;
-  if (!x || !y) return BQ_ERR_NULL;
+  if (!y) return BQ_ERR_NULL;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (K == 0) {
+  if (K == 0) {  // an empty sum: x is not read
     return cudaMemsetAsync(y, 0, (size_t)(M * N * 2), st) == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
   }
+  if (!x) return BQ_ERR_NULL;
   if (!packed || !scales || !zeros) return BQ_ERR_NULL;
   if (!aligned(x, 16) || !aligned(y, 16) || !aligned(packed, 16) || !aligned(scales, 16) || !aligned(zeros, 16))
     return BQ_ERR_ALIGN;

@@ -86,14 +86,14 @@ def test_prefill_deterministic():
     assert torch.equal(y1, y2)
 
 
-@pytest.mark.parametrize("name,N,K,bits", [
-    ("q", 4096, 4096, 4), ("gate", 14336, 4096, 4), ("down", 4096, 14336, 4), ("down", 4096, 14336, 2),
+@pytest.mark.parametrize("name,N,K,bits,M", [
+    ("q", 4096, 4096, 4, 2048), ("gate", 14336, 4096, 4, 2048), ("down", 4096, 14336, 4, 2048),
+    ("down", 4096, 14336, 2, 2048), ("gate", 14336, 4096, 2, 8192), ("qwen_up", 49152, 8192, 4, 2048),
 ])
-def test_prefill_full_size_sampled(name, N, K, bits):
-    """Llama-3-8B projection shapes at 2048 prefill tokens; the oracle checks
-    a sample of output channels and tokens (rows and tokens are independent)."""
+def test_prefill_full_size_sampled(name, N, K, bits, M):
+    """Prefill shapes at the bench's token counts; the oracle checks a sample
+    of output channels and tokens (rows and tokens are independent)."""
     group = 128 if bits == 4 else 64
-    M = 2048
     W = synth.normal((N, K), 0.02, seed=51, dtype="f16", device=DEV)
     x = synth.activations(M, K, seed=52, device=DEV)
     pk, sc, ze = bq.bq_quantize(W, bits, group, "interleaved")
