@@ -450,6 +450,16 @@ def gemm_numbers(Ms, bf16, bf16_sus, reps=10):
     return res
 
 
+def workload_config(args):
+    """The workload both arms report (the reference arm times a bounded sample of it)."""
+    bits = args.bits
+    group = 128 if bits == 4 else 64
+    return {"workload": f"Llama-3-8B-shaped decode stack, {args.layers} layers x 7 projections "
+                        f"(q/k/v and gate/up fused along N: 4 linears per layer), "
+                        f"INT{bits} g{group} weight-only, M in {{1,4,16}} per step",
+            "layers": args.layers, "bits": bits, "group": group, "M": list(M_SET)}
+
+
 def run_gpu(args, world, rank, local):
     hbm, bf16, bf16_sus, peak_kind = peaks()
     bits, group = args.bits, (128 if args.bits == 4 else 64)
@@ -520,10 +530,7 @@ def run_gpu(args, world, rank, local):
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(t_step * 1e3, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": f"bf16 x int{bits} -> fp32 acc", "data": "synthetic",
-        "config": {"workload": f"Llama-3-8B-shaped decode stack, {args.layers} layers x 7 projections "
-                               f"(q/k/v and gate/up fused along N: 4 linears per layer), "
-                               f"INT{bits} g{group} weight-only, M in {{1,4,16}} per step",
-                   "layers": args.layers, "bits": bits, "group": group, "M": list(Ms),
+        "config": {**workload_config(args),
                    "weights": "fp16 N(0,0.02)" if bits == 4 else "fp16 Student-t4 std 0.02 + 0.1% x10 outlier cols",
                    "activations": "bf16 N(0,1)", "l2": "inputs larger than L2 (packed stack %.2f GB)" %
                    (sum(weight_bytes(N, K, bits, group) for (_, _, N, K, _) in stack.fused) / 1e9),
@@ -593,8 +600,7 @@ def run_reference(args, world, rank):
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t * 1e3, 2), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"Llama-3-8B-shaped decode stack, INT{args.bits}, M in {{1,4,16}} "
-                               f"(bounded sample: first {args.oracle_layers} layer(s))"},
+        "config": workload_config(args),
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
                          "sample": f"first {args.oracle_layers} layer(s) x 4 linears (qkv, o, gate_up, down) "
                                    f"x M in {{1,4,16}} per step"},
