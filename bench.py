@@ -15,7 +15,8 @@ Printed: ONE JSON line (rank 0).  ``value`` = effective weight GB/s of the
 whole job = (packed codes + scales + zeros + x + y bytes of every linear of
 the step, over all ranks) / max-over-ranks step time.  Extra fields report
 per-M numbers, per-shape numbers, the quantizer over the whole ~7B-weight
-stack, the prefill GEMM (tcgen05 path, M = 2048 and 8192 tokens against the
+stack and on one 8192x49152 matrix (with the fused fake-quantization pass),
+the prefill GEMM (tcgen05 path, M = 2048 and 8192 tokens against the
 14336x4096, 4096x14336, 49152x8192 and 8192x49152 weights at INT4 and INT2)
 in TFLOP/s, the end-to-end host-buffer path, the roofline of the dominant
 kernel (the decode GEMV) and the CPU oracle baseline.
@@ -410,6 +411,47 @@ def e2e_numbers(stack, Ms, steps, warmup, world):
     return t, h2d, d2h
 
 
+def quant_shape_numbers(hbm, reps=10):
+    """Quantizer and fused fake-quantization on one 8192x49152 fp16 matrix
+    (N(0, 0.02)): GB/s of algorithmic bytes (read 2 B per weight; write
+    codes + scales + zeros, or 2 B per weight for the fake-quantized output)."""
+    N, K = 8192, 49152
+    W = synth.normal((N, K), 0.02, seed=5, dtype="f16", device="cuda")
+    res = {}
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            b.synchronize()
+            ts.append(a.elapsed_time(b) / 1e3)
+        return statistics.median(ts)
+
+    for bits, group in ((4, 128), (2, 64)):
+        out = bq.bq_quantize(W, bits, group, "interleaved")
+        t = timed(lambda: bq.bq_quantize(W, bits, group, "interleaved", out=out))
+        byts = N * K * 2 + weight_bytes(N, K, bits, group)
+        res[f"quantize {N}x{K} INT{bits} g{group}"] = {"us": round(t * 1e6, 1), "GBps": round(byts / t / 1e9, 1),
+                                                       "frac_of_measured_hbm": round(byts / t / 1e9 / hbm, 4)}
+        del out
+    fq = torch.empty_like(W)
+    t = timed(lambda: bq.bq_fake_quantize(W, 4, 128, out=fq))
+    byts = N * K * 4
+    res[f"fake_quantize {N}x{K} INT4 g128 fp16->fp16"] = {"us": round(t * 1e6, 1), "GBps": round(byts / t / 1e9, 1),
+                                                          "frac_of_measured_hbm": round(byts / t / 1e9 / hbm, 4)}
+    del W, fq
+    torch.cuda.empty_cache()
+    if bq.bq_device_status() != bq.BQ_OK:
+        raise RuntimeError("quantizer reported a device error")
+    return res
+
+
 GEMM_SHAPES = ((14336, 4096), (4096, 14336), (49152, 8192), (8192, 49152))
 
 
@@ -516,6 +558,8 @@ def run_gpu(args, world, rank, local):
                 "us_per_launch_avg": round(t_step / launches_per_step * 1e6, 3)}
 
     extra = {"per_M": per_m, "per_shape": shapes, "quantizer_stack": None}
+    if not args.no_quant:
+        extra["quantizer_8192x49152"] = quant_shape_numbers(hbm)
     if not args.no_gemm:
         del g
         extra["prefill_gemm"] = gemm_numbers((2048, 8192) if not args.quick else (2048,), bf16,

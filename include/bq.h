@@ -164,6 +164,24 @@ bq_status bq_dequantize(const void *packed, const float *scales, const uint8_t *
                         void *W_out, bq_dtype otype, void *stream);
 
 /*
+ * bq_fake_quantize: W_out = dequant(quant(W)) in one pass, without storing
+ * codes, scales or zeros -- the forward of quantization-aware training
+ * ("大模型量化实战", section 5.2: a FakeQuantize module simulates
+ * round(x/s) + z in the forward pass; "A Survey of Low-bit Large Language
+ * Models", section 8.1).
+ *   W       [rows, cols] of wtype (BQ_F16 / BQ_BF16), 16-byte aligned
+ *   groups  `group` consecutive elements along cols (cols % group == 0;
+ *           group in {8, 16, 32, 64, 128, 256}); bits 2 or 4
+ *   W_out   [rows, cols] of otype (BQ_F16, BQ_BF16 or BQ_F32), 16-byte aligned;
+ *           element (q - z) * s computed in fp32 and rounded once to otype, so
+ *           W_out equals bq_dequantize(bq_quantize(W)) bit for bit
+ * A non-finite weight sets BQ_ERR_NONFINITE in the device status (its group's
+ * outputs are unspecified).
+ */
+bq_status bq_fake_quantize(const void *W, bq_dtype wtype, int64_t rows, int64_t cols, int bits, int group,
+                           void *W_out, bq_dtype otype, void *stream);
+
+/*
  * bq_linear: y[M, N] = x[M, K] . dequant(W)^T.
  *   x        [M, K] of xtype (BQ_BF16 or BQ_F16), 16-byte aligned rows (K % 8 == 0)
  *   packed / scales / zeros: from bq_quantize in BQ_LAYOUT_INTERLEAVED; all

@@ -32,7 +32,7 @@ GROUP_OF_BITS = {4: 128, 2: 64}
 #: every symbol include/bq.h declares
 EXPORTS = (
     "bq_packed_bytes", "bq_group_count", "bq_mixed_offsets", "bq_quantize", "bq_quantize_mixed",
-    "bq_dequantize", "bq_linear", "bq_check_division", "bq_set_option", "bq_get_option", "bq_device_status",
+    "bq_dequantize", "bq_fake_quantize", "bq_linear", "bq_check_division", "bq_set_option", "bq_get_option", "bq_device_status",
     "bq_status_string", "bq_version",
 )
 BQ_OPT_LINEAR_OVERLAP = 0
@@ -70,6 +70,8 @@ def lib(path: str | None = None):
     L.bq_quantize_mixed.restype = i32
     L.bq_dequantize.argtypes = [vp, vp, vp, vp, i32, i32, i64, i64, i32, vp, i32, vp]
     L.bq_dequantize.restype = i32
+    L.bq_fake_quantize.argtypes = [vp, i32, i64, i64, i32, i32, vp, i32, vp]
+    L.bq_fake_quantize.restype = i32
     L.bq_linear.argtypes = [vp, i32, i64, i64, vp, vp, vp, vp, i32, i32, i64, i32, vp, vp]
     L.bq_linear.restype = i32
     L.bq_check_division.argtypes = [ctypes.c_uint32, ctypes.c_uint32, i32, vp, vp]
@@ -181,6 +183,17 @@ def bq_dequantize(packed, scales, zeros, rows: int, cols: int, bits: int = 4, gr
                              rows, cols, LAYOUTS[layout], _ptr(out), DTYPE_CODE[out_dtype], _stream(stream))
     _check("bq_dequantize", st)
     return out
+
+
+def bq_fake_quantize(W: torch.Tensor, bits: int, group: int | None = None, out_dtype=None, out=None, stream=None):
+    """dequant(quant(W)) in one pass (codes, scales, zeros not stored); out in W's dtype by default."""
+    group = group or GROUP_OF_BITS[bits]
+    N, K = W.shape
+    o = out if out is not None else torch.empty((N, K), dtype=out_dtype or W.dtype, device=W.device)
+    st = lib().bq_fake_quantize(_ptr(W), DTYPE_CODE[W.dtype], N, K, bits, group, _ptr(o), DTYPE_CODE[o.dtype],
+                                _stream(stream))
+    _check("bq_fake_quantize", st)
+    return o
 
 
 def bq_linear(x: torch.Tensor, packed, scales, zeros, N: int, bits: int = 4, group: int | None = None,

@@ -9,6 +9,7 @@
 #include "../../include/bq.h"
 #include "common.cuh"
 #include "dequant.cuh"
+#include "fakequant.cuh"
 #include "gemm.cuh"
 #include "gemv.cuh"
 #include "quantize.cuh"
@@ -147,6 +148,29 @@ bq_status quantize_tiled(const uint16_t *W, int64_t N, int64_t K, int group, uin
     case 256: return quantize_tma<WT, BITS, 256>(W, N, K, packed, scales, zeros, st);
     default: return BQ_ERR_UNSUPPORTED;
   }
+}
+
+template <int WT, int OT, int BITS>
+bq_status fake_quant_dispatch(const uint16_t *W, int64_t elems, int group, void *out, cudaStream_t st) {
+  using T = typename OutT<OT>::T;
+  const int64_t grid = grid_for((elems + 255) / 256);
+  T *o = reinterpret_cast<T *>(out);
+#define BQ_FQ(G_)                                                                           \
+  case G_:                                                                                  \
+    fake_quant_kernel<WT, OT, BITS, G_, 2><<<grid, kThreads, 0, st>>>(W, elems, o);          \
+    break;
+  switch (group) {
+    BQ_FQ(8) BQ_FQ(16) BQ_FQ(32) BQ_FQ(64) BQ_FQ(128) BQ_FQ(256)
+    default: return BQ_ERR_UNSUPPORTED;
+  }
+#undef BQ_FQ
+  return launch_status();
+}
+
+template <int WT, int OT>
+bq_status fake_quant_bits(const uint16_t *W, int64_t elems, int bits, int group, void *out, cudaStream_t st) {
+  return bits == 4 ? fake_quant_dispatch<WT, OT, 4>(W, elems, group, out, st)
+                   : fake_quant_dispatch<WT, OT, 2>(W, elems, group, out, st);
 }
 
 bool canonical_group_ok(int g) { return g == 8 || g == 16 || g == 32 || g == 64 || g == 128 || g == 256; }
@@ -556,6 +580,29 @@ bq_status bq_dequantize(const void *packed, const float *scales, const uint8_t *
   if (otype == BQ_F16) return dequant_uniform<0>(pk, scales, zeros, bits, group, rows, cols, layout, W_out, st);
   if (otype == BQ_BF16) return dequant_uniform<1>(pk, scales, zeros, bits, group, rows, cols, layout, W_out, st);
   return dequant_uniform<2>(pk, scales, zeros, bits, group, rows, cols, layout, W_out, st);
+}
+
+bq_status bq_fake_quantize(const void *W, bq_dtype wtype, int64_t rows, int64_t cols, int bits, int group,
+                           void *W_out, bq_dtype otype, void *stream) {
+  if (rows < 0 || cols < 0) return BQ_ERR_SHAPE;
+  if (wtype != BQ_F16 && wtype != BQ_BF16) return BQ_ERR_UNSUPPORTED;
+  if (otype != BQ_F16 && otype != BQ_BF16 && otype != BQ_F32) return BQ_ERR_UNSUPPORTED;
+  if (!valid_bits(bits) || !canonical_group_ok(group)) return BQ_ERR_UNSUPPORTED;
+  if (cols % group) return BQ_ERR_SHAPE;
+  if (rows == 0 || cols == 0) return BQ_OK;
+  if (!W || !W_out) return BQ_ERR_NULL;
+  if (!aligned(W, 16) || !aligned(W_out, 16)) return BQ_ERR_ALIGN;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const uint16_t *w = reinterpret_cast<const uint16_t *>(W);
+  const int64_t elems = rows * cols;
+  if (wtype == BQ_F16) {
+    if (otype == BQ_F16) return fake_quant_bits<0, 0>(w, elems, bits, group, W_out, st);
+    if (otype == BQ_BF16) return fake_quant_bits<0, 1>(w, elems, bits, group, W_out, st);
+    return fake_quant_bits<0, 2>(w, elems, bits, group, W_out, st);
+  }
+  if (otype == BQ_F16) return fake_quant_bits<1, 0>(w, elems, bits, group, W_out, st);
+  if (otype == BQ_BF16) return fake_quant_bits<1, 1>(w, elems, bits, group, W_out, st);
+  return fake_quant_bits<1, 2>(w, elems, bits, group, W_out, st);
 }
 
 bq_status bq_linear(const void *x, bq_dtype xtype, int64_t M, int64_t K, const void *packed, const float *scales,

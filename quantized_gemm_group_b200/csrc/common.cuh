@@ -262,6 +262,16 @@ BQ_DEV bool mbar_test_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// One 2D tensor-map (TMA) tile load into this CTA's shared memory,
+// completing on `bar`; coordinates (c0 innermost, c1) in elements.
+BQ_DEV void tma_load_2d(uint32_t dst, const CUtensorMap *map, int c0, int c1, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+
 // Bounded wait on the phase with the given parity: false after `limit` polls.
 constexpr uint32_t kWaitLimit = 1u << 22;
 BQ_DEV bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t limit = kWaitLimit) {

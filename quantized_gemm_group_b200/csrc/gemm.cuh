@@ -200,13 +200,6 @@ BQ_DEV void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 template <uint32_t N> BQ_DEV void setmaxnreg_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
 template <uint32_t N> BQ_DEV void setmaxnreg_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
 
-BQ_DEV void tma_load_2d(uint32_t dst, const CUtensorMap *map, int c0, int c1, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
-      "[%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
-      : "memory");
-}
 
 // Byte offset of bf16 element (row, k) of a 128-byte-swizzled K-major tile
 // (rows of 64 elements; the 16-byte chunk index is XORed with row % 8).

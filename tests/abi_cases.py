@@ -85,6 +85,20 @@ def test_linear_validation(L):
     assert lin(L, M=0, x=None, y=None) == bq.BQ_OK
 
 
+def test_fake_quantize_validation(L):
+    f = L.bq_fake_quantize
+    assert f(FAKE, bq.BQ_F32, 16, 128, 4, 128, FAKE, bq.BQ_BF16, None) == bq.BQ_ERR_UNSUPPORTED  # W must be 16-bit
+    assert f(FAKE, bq.BQ_F16, 16, 128, 4, 128, FAKE, 7, None) == bq.BQ_ERR_UNSUPPORTED
+    assert f(FAKE, bq.BQ_F16, 16, 128, 3, 128, FAKE, bq.BQ_F32, None) == bq.BQ_ERR_UNSUPPORTED
+    assert f(FAKE, bq.BQ_F16, 16, 128, 4, 96, FAKE, bq.BQ_F32, None) == bq.BQ_ERR_UNSUPPORTED
+    assert f(FAKE, bq.BQ_F16, 16, 192, 4, 128, FAKE, bq.BQ_F32, None) == bq.BQ_ERR_SHAPE   # cols % group
+    assert f(FAKE, bq.BQ_F16, -1, 128, 4, 128, FAKE, bq.BQ_F32, None) == bq.BQ_ERR_SHAPE
+    assert f(None, bq.BQ_F16, 16, 128, 4, 128, FAKE, bq.BQ_F32, None) == bq.BQ_ERR_NULL
+    assert f(FAKE_MIS, bq.BQ_F16, 16, 128, 4, 128, FAKE, bq.BQ_F32, None) == bq.BQ_ERR_ALIGN
+    assert f(FAKE, bq.BQ_F16, 16, 128, 4, 128, FAKE_MIS, bq.BQ_F32, None) == bq.BQ_ERR_ALIGN
+    assert f(None, bq.BQ_F16, 0, 128, 4, 128, None, bq.BQ_F32, None) == bq.BQ_OK
+
+
 def test_dequant_validation(L):
     f = L.bq_dequantize
     assert f(FAKE, FAKE, FAKE, None, 4, 128, 16, 128, 1, FAKE, 7, None) == bq.BQ_ERR_UNSUPPORTED
