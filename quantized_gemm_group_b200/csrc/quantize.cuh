@@ -11,12 +11,12 @@
 //     the thread writes its 8 codes as one 32-bit (4-bit) or 16-bit (2-bit)
 //     word; scales / zeros row-major [rows, cols/g].
 //   * interleaved layout: a warp owns a unit of 16 rows x U columns
-//     (U = max(tile width, g)); lane L loads exactly the weights whose codes
+//     (U = max(tile width, g)); lane L takes exactly the weights whose codes
 //     form its own 16-byte slot of each 512-byte tile, so no permutation pass
 //     is needed; groups are reduced over the 4 lanes sharing a row; tiles and
 //     scales / zeros go to their 128-row-block-major places (il_tile_offset,
-//     il_meta_index).  The next unit's weights are loaded before the current
-//     one is computed.
+//     il_meta_index).  A producer warp stages the weights by TMA
+//     (quantize_tma_kernel); mixed maps load them per lane (load_unit).
 // The per-element arithmetic runs on packed f32x2 operations (two elements
 // per instruction); the clamp to 2^b - 1 is only evaluated in groups whose
 // largest element needs it.
@@ -244,48 +244,11 @@ BQ_DEV bool quantize_unit(const UnitRegs<BITS, G> &u, int64_t N, int64_t K, int6
   return bad_any;
 }
 
-template <int WT, int BITS, int G>
-__global__ void __launch_bounds__(256)
-quantize_tiled_kernel(const uint16_t *__restrict__ W, int64_t N, int64_t K,
-                      uint8_t *__restrict__ packed, float *__restrict__ scales,
-                      uint8_t *__restrict__ zeros) {
-  using UG = UnitGeom<BITS, G>;
-  const int lane = threadIdx.x & 31;
-  const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  const int64_t ku = K / UG::U;
-  const int64_t units = (N / 16) * ku;
-  bool bad = false;
-  UnitRegs<BITS, G> ua, ub;
-  auto at = [&](int64_t u, int64_t *row0, int64_t *col0) {
-    const int64_t rb = u / ku;
-    *row0 = rb * 16;
-    *col0 = (u - rb * ku) * UG::U;
-  };
-  int64_t r0, c0;
-  int64_t u = warp;
-  if (u < units) { at(u, &r0, &c0); load_unit(ua, W, K, r0, c0, lane); }
-  for (; u < units; u += 2 * nwarps) {
-    const int64_t u1 = u + nwarps;
-    int64_t r1, c1;
-    if (u1 < units) { at(u1, &r1, &c1); load_unit(ub, W, K, r1, c1, lane); }
-    at(u, &r0, &c0);
-    bad |= quantize_unit<WT, BITS, G>(ua, N, K, r0, c0, packed, scales, zeros, lane);
-    if (u1 < units) {
-      const int64_t u2 = u1 + nwarps;
-      int64_t r2, c2;
-      if (u2 < units) { at(u2, &r2, &c2); load_unit(ua, W, K, r2, c2, lane); }
-      bad |= quantize_unit<WT, BITS, G>(ub, N, K, r1, c1, packed, scales, zeros, lane);
-    }
-  }
-  if (bad) bq_flag(BQ_FLAG_NONFINITE);
-}
-
 // ---------------------------------------------------------------------------
 // interleaved layout, weights staged by TMA
 // ---------------------------------------------------------------------------
-// The same per-unit arithmetic and stores as quantize_tiled_kernel, with the
-// weights brought into shared memory by TMA instead of held in registers:
+// Per unit the arithmetic and stores of quantize_unit, with the weights
+// brought into shared memory by TMA rather than loaded into registers:
 // a super-unit is 64 rows x U columns (four 16-row units), loaded as U / 64
 // boxes of 64 columns x 64 rows with the 128-byte swizzle (16-byte chunk c
 // of row r stored at chunk c ^ (r % 8)), which makes each lane's 4-byte
