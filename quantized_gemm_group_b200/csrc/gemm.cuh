@@ -424,12 +424,17 @@ BQ_DEV void gemm_epilogue(const GemmArgs &a, const float *sc, int e, int warp, i
     if (g + 1 < ngroups) s_next = __ldg(sc + (int64_t)(g + 1) * 128 + rloc);
     if (!mbar_wait(d_full + 8u * buf, (g >> 1) & 1)) { *abort = 1; bq_flag(BQ_FLAG_TIMEOUT); ok = false; break; }
     tc_fence_after();
+    const float2 s2 = make_float2(s, s);
 #pragma unroll
     for (int cc = 0; cc < 4; ++cc) {
       float v[16];
       tmem_ld16(tmem + lane_addr + (uint32_t)(buf * kGemmTokTile + col0 + cc * 16), v);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) acc[cc * 16 + i] = __fmaf_rn(s, v[i], acc[cc * 16 + i]);
+      for (int i = 0; i < 16; i += 2) {  // packed fp32x2 FMA: two columns per instruction
+        const float2 r = __ffma2_rn(s2, make_float2(v[i], v[i + 1]), make_float2(acc[cc * 16 + i], acc[cc * 16 + i + 1]));
+        acc[cc * 16 + i] = r.x;
+        acc[cc * 16 + i + 1] = r.y;
+      }
     }
     tc_fence_before();
     __syncwarp();
