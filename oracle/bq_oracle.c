@@ -138,14 +138,67 @@ int bqo_quantize_group(const float *x, int g, int bits,
     return BQO_OK;
 }
 
+/* Symmetric abs-max scheme ("大模型量化实战", section 2.3: s = x_absmax /
+ * (2^(b-1) - 1) -- 127 at 8 bits -- and z fixed at 0, codes round(x / s)).
+ * Readings: applied per group like the MinMax scheme; codes are stored
+ * offset by 2^(b-1) (z = 2^(b-1)) so that the unsigned storage and
+ * dequant(q) = (q - z) * s of the MinMax scheme apply unchanged; the same
+ * rounding as R3 (one fp32 division, half to even); an all-zero group
+ * stores s = 0 and every code equal to z.
+ *   s = max |x| / (2^(b-1) - 1)
+ *   q = clamp(round(x / s) + 2^(b-1), 0, 2^b - 1)                            */
+int bqo_quantize_group_sym(const float *x, int g, int bits,
+                           float *s_out, int *z_out, uint8_t *q_out)
+{
+    if (g <= 0 || bits < 2 || bits > 8) return BQO_ERR_ARG;
+    const int qmax = (1 << bits) - 1;
+    const int z = 1 << (bits - 1);
+
+    float amax = 0.0f;
+    for (int i = 0; i < g; ++i) {
+        if (!isfinite(x[i])) return BQO_ERR_NONFINITE;
+        float a = fabsf(x[i]);
+        if (a > amax) amax = a;
+    }
+    float s = amax / (float)(z - 1);
+    if (!isfinite(s)) return BQO_ERR_NONFINITE;
+    if (s == 0.0f) {
+        *s_out = 0.0f;
+        *z_out = z;
+        memset(q_out, z, (size_t)g);
+        return BQO_OK;
+    }
+    for (int i = 0; i < g; ++i) {
+        int q = (int)nearbyintf(x[i] / s) + z;
+        q_out[i] = (uint8_t)(q < 0 ? 0 : (q > qmax ? qmax : q));
+    }
+    *s_out = s;
+    *z_out = z;
+    return BQO_OK;
+}
+
 /* Whole matrix W[rows, cols] (row-major, fp16 when wtype == 0, bf16 when
  * wtype == 1), groups of `group` consecutive elements along cols (R5).
  * Only rows [r0, r1) are processed so that callers may split rows across
  * threads.  Outputs: codes[rows*cols] unpacked, scales/zeros[rows*(cols/group)]. */
+int bqo_quantize_scheme(const uint16_t *W, int wtype, int64_t rows, int64_t cols,
+                        int bits, int group, int scheme, int64_t r0, int64_t r1,
+                        uint8_t *codes, float *scales, uint8_t *zeros);
+
 int bqo_quantize(const uint16_t *W, int wtype, int64_t rows, int64_t cols,
                  int bits, int group, int64_t r0, int64_t r1,
                  uint8_t *codes, float *scales, uint8_t *zeros)
 {
+    return bqo_quantize_scheme(W, wtype, rows, cols, bits, group, 0, r0, r1, codes, scales, zeros);
+}
+
+/* scheme 0: asymmetric MinMax (bqo_quantize_group); 1: symmetric abs-max
+ * (bqo_quantize_group_sym). */
+int bqo_quantize_scheme(const uint16_t *W, int wtype, int64_t rows, int64_t cols,
+                        int bits, int group, int scheme, int64_t r0, int64_t r1,
+                        uint8_t *codes, float *scales, uint8_t *zeros)
+{
+    if (scheme != 0 && scheme != 1) return BQO_ERR_ARG;
     if (group <= 0 || cols % group != 0 || r0 < 0 || r1 > rows) return BQO_ERR_ARG;
     if (group > 4096) return BQO_ERR_ARG;
     if (fegetround() != FE_TONEAREST) return BQO_ERR_ARG;
@@ -157,8 +210,8 @@ int bqo_quantize(const uint16_t *W, int wtype, int64_t rows, int64_t cols,
             for (int i = 0; i < group; ++i) buf[i] = decode(src[i], wtype);
             float s;
             int z;
-            int rc = bqo_quantize_group(buf, group, bits, &s, &z,
-                                        codes + n * cols + j * group);
+            int rc = scheme ? bqo_quantize_group_sym(buf, group, bits, &s, &z, codes + n * cols + j * group)
+                            : bqo_quantize_group(buf, group, bits, &s, &z, codes + n * cols + j * group);
             if (rc) return rc;
             scales[n * G + j] = s;
             zeros[n * G + j] = (uint8_t)z;

@@ -54,6 +54,10 @@ def lib():
             L.bqo_quantize_group.restype = i32
             L.bqo_quantize.argtypes = [vp, i32, i64, i64, i32, i32, i64, i64, vp, vp, vp]
             L.bqo_quantize.restype = i32
+            L.bqo_quantize_scheme.argtypes = [vp, i32, i64, i64, i32, i32, i32, i64, i64, vp, vp, vp]
+            L.bqo_quantize_scheme.restype = i32
+            L.bqo_quantize_group_sym.argtypes = [vp, i32, i32, vp, vp, vp]
+            L.bqo_quantize_group_sym.restype = i32
             L.bqo_code_position.argtypes = [i32, i64, i64, i64, i64, i32, vp, vp]
             L.bqo_code_position.restype = None
             L.bqo_pack.argtypes = [vp, i64, i64, i32, i32, vp]
@@ -132,20 +136,25 @@ def _row_chunks(rows: int, threads: int):
 # quantizer
 # ---------------------------------------------------------------------------
 
-def quantize_group(x: np.ndarray, bits: int):
+def quantize_group(x: np.ndarray, bits: int, scheme: str = "asymmetric"):
     """One group of fp32 values -> (s, z, q)."""
     x = np.ascontiguousarray(x, dtype=np.float32)
     q = np.zeros(x.size, dtype=np.uint8)
     s = ctypes.c_float()
     z = ctypes.c_int()
-    rc = lib().bqo_quantize_group(_p(x), x.size, bits, ctypes.byref(s), ctypes.byref(z), _p(q))
+    fn = lib().bqo_quantize_group_sym if scheme == "symmetric" else lib().bqo_quantize_group
+    rc = fn(_p(x), x.size, bits, ctypes.byref(s), ctypes.byref(z), _p(q))
     if rc:
         raise OracleError(f"bqo_quantize_group rc={rc}")
     return float(np.float32(s.value)), int(z.value), q
 
 
-def quantize(w_bits: np.ndarray, wtype: str, bits: int, group: int, threads: int = 1):
-    """Quantize W (uint16 bit patterns of fp16/bf16, shape [N, K]).
+SCHEMES = {"asymmetric": 0, "symmetric": 1}
+
+
+def quantize(w_bits: np.ndarray, wtype: str, bits: int, group: int, threads: int = 1, scheme: str = "asymmetric"):
+    """Quantize W (uint16 bit patterns of fp16/bf16, shape [N, K]) with the
+    asymmetric MinMax scheme (default) or the symmetric abs-max scheme.
 
     Returns unpacked codes u8 [N, K], scales f32 [N, K/group], zeros u8 [N, K/group].
     """
@@ -160,8 +169,8 @@ def quantize(w_bits: np.ndarray, wtype: str, bits: int, group: int, threads: int
     L = lib()
 
     def run(r):
-        return L.bqo_quantize(_p(w_bits), WTYPE[wtype], N, K, bits, group, r[0], r[1],
-                              _p(codes), _p(scales), _p(zeros))
+        return L.bqo_quantize_scheme(_p(w_bits), WTYPE[wtype], N, K, bits, group, SCHEMES[scheme], r[0], r[1],
+                                     _p(codes), _p(scales), _p(zeros))
 
     if threads <= 1:
         rcs = [run((0, N))]

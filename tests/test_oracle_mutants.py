@@ -33,6 +33,10 @@ MUTANTS = {
     "tile_order_row_major": ("*byte_off = block_start + (kt * Rb + t) * 512", "*byte_off = block_start + (t * (cols / T) + kt) * 512"),
     "f16_bias": ("mag = ldexpf((float)(1024 + f), e - 25);", "mag = ldexpf((float)(1024 + f), e - 24);"),
     "f16_subnormal": ("mag = ldexpf((float)f, -24);", "mag = ldexpf((float)f, -25);"),
+    "sym_levels_2^b-1": ("float s = amax / (float)(z - 1);", "float s = amax / (float)qmax;"),
+    "sym_no_offset": ("int q = (int)nearbyintf(x[i] / s) + z;", "int q = (int)nearbyintf(x[i] / s);"),
+    "sym_round_half_away": ("int q = (int)nearbyintf(x[i] / s) + z;", "int q = (int)roundf(x[i] / s) + z;"),
+    "sym_min_not_abs": ("float a = fabsf(x[i]);", "float a = x[i];"),
 }
 
 # cheap pins first; each mutant only has to fail one of them
@@ -50,6 +54,9 @@ PINS = [
     (P.test_linear_closed_form, {"bits": 4, "g": 128}),
     (P.test_brute_force_optimal_codes, {"bits": 2}),
     (P.test_exact_rational_arithmetic, {}),
+    (P.test_sym_worked_examples, {"name": "sym_int4_g8_worked.txt"}),
+    (P.test_sym_worked_examples, {"name": "sym_int2_g8_worked.txt"}),
+    (P.test_sym_page_scale_example, {}),
 ]
 
 

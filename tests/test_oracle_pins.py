@@ -441,3 +441,84 @@ def test_interleaved_stacks_whole_blocks(bits):
     pieces = [O.pack_meta(s, z, "interleaved") for s, z in zip(scales, zeros)]
     assert (ms.view(np.uint32) == np.concatenate([p[0] for p in pieces]).view(np.uint32)).all()
     assert (mz == np.concatenate([p[1] for p in pieces])).all()
+
+
+# --------------------------------------------------------------------------
+# symmetric abs-max scheme ("大模型量化实战", section 2.3)
+# --------------------------------------------------------------------------
+
+def exact_group_sym(x32: np.ndarray, bits: int):
+    """The symmetric scheme's steps in exact rational arithmetic."""
+    qmax, zc = (1 << bits) - 1, 1 << (bits - 1)
+    xs = [Fraction(float(v)) for v in x32]
+    amax = max(abs(v) for v in xs)
+    s = rne_f32(amax / (zc - 1))
+    if s == 0:
+        return 0.0, zc, [zc] * len(xs)
+    q = [min(max(rne_int(rne_f32(v / s)) + zc, 0), qmax) for v in xs]
+    return float(s), zc, q
+
+
+@pytest.mark.parametrize("name", ["sym_int4_g8_worked.txt", "sym_int2_g8_worked.txt"])
+def test_sym_worked_examples(name):
+    g = read_golden(name)
+    bits = int(g["bits"][0])
+    x = np.array([float(v) for v in g["x"]], dtype=np.float32)
+    s, z, q = O.quantize_group(x, bits, scheme="symmetric")
+    assert s == float(g["s"][0])
+    assert z == int(g["z"][0])
+    assert q.tolist() == [int(v) for v in g["q"]]
+    assert ((q.astype(np.float64) - z) * s).tolist() == [float(v) for v in g["dequant"]]
+    for key in ("canonical_word32", "canonical_word16"):
+        if key in g:
+            packed = O.pack(q.reshape(1, -1), bits, "canonical")
+            assert int.from_bytes(packed.tobytes(), "little") == int(g[key][0], 16)
+
+
+def test_sym_page_scale_example():
+    """The page's 8-bit example: x_absmax = 5.0 gives s = 5.0 / 127 ~ 0.039."""
+    x = np.array([-5.0, -0.1, 0.0, 0.05, 0.1, 1.0, 2.5, 4.0], dtype=np.float32)
+    s, z, q = O.quantize_group(x, 8, scheme="symmetric")
+    assert s == float(np.float32(5.0) / np.float32(127.0))
+    assert abs(s - 0.039) < 5e-4
+    assert z == 128 and int(q[0]) == 1 and int(q[2]) == 128
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_sym_invariants(bits):
+    rng = np.random.default_rng(7 + bits)
+    for trial in range(300):
+        x = (rng.standard_normal(32) * rng.choice([1e-3, 0.02, 1.0, 30.0])).astype(np.float32)
+        s, z, q = O.quantize_group(x, bits, scheme="symmetric")
+        assert z == 1 << (bits - 1)
+        assert q.min() >= 1 and q.max() <= (1 << bits) - 1       # the code 0 is never needed
+        err = np.abs(x.astype(np.float64) - (q.astype(np.float64) - z) * s)
+        assert err.max() <= s / 2 * (1 + 2.0 ** -20)
+        # round half to even is odd-symmetric: negating the group negates q - z
+        s2, z2, q2 = O.quantize_group(-x, bits, scheme="symmetric")
+        assert s2 == s and ((q2.astype(int) - z2) == -(q.astype(int) - z)).all()
+
+
+def test_sym_exact_rational_arithmetic():
+    rng = np.random.default_rng(11)
+    for bits in (2, 4, 8):
+        for _ in range(200):
+            x = (rng.standard_normal(16) * 0.02).astype(np.float16).astype(np.float32)
+            s, z, q = O.quantize_group(x, bits, scheme="symmetric")
+            es, ez, eq = exact_group_sym(x, bits)
+            assert s == es and z == ez and q.tolist() == eq
+
+
+def test_sym_all_zero_group():
+    s, z, q = O.quantize_group(np.zeros(64, dtype=np.float32), 4, scheme="symmetric")
+    assert s == 0.0 and z == 8 and (q == 8).all()
+
+
+def test_sym_matrix_matches_groups():
+    rng = np.random.default_rng(3)
+    W = (rng.standard_normal((4, 256)) * 0.02).astype(np.float16)
+    codes, scales, zeros = O.quantize(W.view(np.uint16), "f16", 4, 64, scheme="symmetric")
+    for n in range(4):
+        for j in range(4):
+            s, z, q = O.quantize_group(W[n, 64 * j:64 * (j + 1)].astype(np.float32), 4, scheme="symmetric")
+            assert scales[n, j] == s and zeros[n, j] == z and (codes[n, 64 * j:64 * (j + 1)] == q).all()
