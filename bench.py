@@ -440,6 +440,12 @@ def quant_shape_numbers(hbm, reps=10):
         res[f"quantize {N}x{K} INT{bits} g{group}"] = {"us": round(t * 1e6, 1), "GBps": round(byts / t / 1e9, 1),
                                                        "frac_of_measured_hbm": round(byts / t / 1e9 / hbm, 4)}
         del out
+    out = bq.bq_quantize(W, 4, 128, "interleaved", scheme="symmetric")
+    t = timed(lambda: bq.bq_quantize(W, 4, 128, "interleaved", out=out, scheme="symmetric"))
+    byts = N * K * 2 + weight_bytes(N, K, 4, 128)
+    res[f"quantize_symmetric {N}x{K} INT4 g128"] = {"us": round(t * 1e6, 1), "GBps": round(byts / t / 1e9, 1),
+                                                   "frac_of_measured_hbm": round(byts / t / 1e9 / hbm, 4)}
+    del out
     fq = torch.empty_like(W)
     t = timed(lambda: bq.bq_fake_quantize(W, 4, 128, out=fq))
     byts = N * K * 4

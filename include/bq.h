@@ -164,6 +164,20 @@ bq_status bq_dequantize(const void *packed, const float *scales, const uint8_t *
                         void *W_out, bq_dtype otype, void *stream);
 
 /*
+ * bq_quantize_symmetric: the symmetric abs-max scheme ("大模型量化实战",
+ * section 2.3: s = x_absmax / 127 at 8 bits, zero point fixed at 0), per
+ * group like bq_quantize:
+ *     s = max |x| / (2^(b-1) - 1)          fp32, one IEEE division
+ *     q = round(x / s) + 2^(b-1)           half to even; 1 <= q <= 2^b - 1
+ *     z = 2^(b-1) (stored in `zeros`, so dequant(q) = (q - z) * s as above)
+ *     an all-zero group stores s = 0 and every code equal to z
+ * Same arguments, layouts, outputs and errors as bq_quantize; the result is
+ * consumed unchanged by bq_dequantize and bq_linear.
+ */
+bq_status bq_quantize_symmetric(const void *W, bq_dtype wtype, int64_t rows, int64_t cols, int bits, int group,
+                                bq_layout layout, void *packed, float *scales, uint8_t *zeros, void *stream);
+
+/*
  * bq_fake_quantize: W_out = dequant(quant(W)) in one pass, without storing
  * codes, scales or zeros -- the forward of quantization-aware training
  * ("大模型量化实战", section 5.2: a FakeQuantize module simulates

@@ -31,7 +31,8 @@ GROUP_OF_BITS = {4: 128, 2: 64}
 
 #: every symbol include/bq.h declares
 EXPORTS = (
-    "bq_packed_bytes", "bq_group_count", "bq_mixed_offsets", "bq_quantize", "bq_quantize_mixed",
+    "bq_packed_bytes", "bq_group_count", "bq_mixed_offsets", "bq_quantize", "bq_quantize_symmetric",
+    "bq_quantize_mixed",
     "bq_dequantize", "bq_fake_quantize", "bq_linear", "bq_check_division", "bq_set_option", "bq_get_option", "bq_device_status",
     "bq_status_string", "bq_version",
 )
@@ -66,6 +67,8 @@ def lib(path: str | None = None):
     L.bq_mixed_offsets.restype = i32
     L.bq_quantize.argtypes = [vp, i32, i64, i64, i32, i32, i32, vp, vp, vp, vp]
     L.bq_quantize.restype = i32
+    L.bq_quantize_symmetric.argtypes = [vp, i32, i64, i64, i32, i32, i32, vp, vp, vp, vp]
+    L.bq_quantize_symmetric.restype = i32
     L.bq_quantize_mixed.argtypes = [vp, i32, i64, i64, vp, i32, vp, vp, vp, vp]
     L.bq_quantize_mixed.restype = i32
     L.bq_dequantize.argtypes = [vp, vp, vp, vp, i32, i32, i64, i64, i32, vp, i32, vp]
@@ -137,9 +140,10 @@ def bq_mixed_offsets(bit_map, rows: int, cols: int):
 # ---------------------------------------------------------------------------
 
 def bq_quantize(W: torch.Tensor, bits: int, group: int | None = None, layout: str = "interleaved",
-                out=None, stream=None):
-    """Quantize W [N, K] (fp16/bf16, CUDA).  Returns (packed u8, scales f32, zeros u8): scales / zeros
-    are [N, K/g] in the canonical layout and flat (16-row-block-major order) in the interleaved one."""
+                out=None, stream=None, scheme: str = "asymmetric"):
+    """Quantize W [N, K] (fp16/bf16, CUDA) with the asymmetric MinMax scheme (default) or the
+    symmetric abs-max one.  Returns (packed u8, scales f32, zeros u8): scales / zeros are [N, K/g]
+    in the canonical layout and flat (128-row-block-major order) in the interleaved one."""
     group = group or GROUP_OF_BITS[bits]
     N, K = W.shape
     if out is None:
@@ -149,8 +153,9 @@ def bq_quantize(W: torch.Tensor, bits: int, group: int | None = None, layout: st
         zeros = torch.empty(mshape, dtype=torch.uint8, device=W.device)
     else:
         packed, scales, zeros = out
-    st = lib().bq_quantize(_ptr(W), DTYPE_CODE[W.dtype], N, K, bits, group, LAYOUTS[layout],
-                           _ptr(packed), _ptr(scales), _ptr(zeros), _stream(stream))
+    fn = lib().bq_quantize_symmetric if scheme == "symmetric" else lib().bq_quantize
+    st = fn(_ptr(W), DTYPE_CODE[W.dtype], N, K, bits, group, LAYOUTS[layout],
+            _ptr(packed), _ptr(scales), _ptr(zeros), _stream(stream))
     _check("bq_quantize", st)
     return packed, scales, zeros
 

@@ -93,13 +93,13 @@ int tile_width(int bits) { return bits == 4 ? 64 : 128; }
 // quantize dispatch
 // ---------------------------------------------------------------------------
 
-template <int WT, int BITS>
+template <int WT, int BITS, int SCHEME>
 bq_status quantize_canonical(const uint16_t *W, int64_t elems, int group, uint8_t *packed, float *scales,
                              uint8_t *zeros, cudaStream_t st) {
   const int64_t grid = grid_for((elems + 255) / 256);
 #define BQ_QC(G)                                                                              \
   case G:                                                                                     \
-    quantize_canonical_kernel<WT, BITS, G, 4><<<grid, kThreads, 0, st>>>(W, elems, packed, scales, zeros); \
+    quantize_canonical_kernel<WT, BITS, G, 4, SCHEME><<<grid, kThreads, 0, st>>>(W, elems, packed, scales, zeros); \
     break;
   switch (group) {
     BQ_QC(8) BQ_QC(16) BQ_QC(32) BQ_QC(64) BQ_QC(128) BQ_QC(256)
@@ -111,13 +111,13 @@ bq_status quantize_canonical(const uint16_t *W, int64_t elems, int group, uint8_
 
 // Interleaved layout: the TMA-staged kernel, two CTAs per SM, each with a ring
 // of super-units (64 rows x U columns) in about 110 KB of shared memory.
-template <int WT, int BITS, int G>
+template <int WT, int BITS, int G, int SCHEME>
 bq_status quantize_tma(const uint16_t *W, int64_t N, int64_t K, uint8_t *packed, float *scales, uint8_t *zeros,
                        cudaStream_t st) {
   constexpr int U = UnitGeom<BITS, G>::U;
   constexpr int SU = (U / 64) * 8192;
   constexpr int kBudget = 113 * 1024;
-  auto kern = quantize_tma_kernel<WT, BITS, G>;
+  auto kern = quantize_tma_kernel<WT, BITS, G, SCHEME>;
   static bool attr_set = false;
   if (!attr_set) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kBudget) != cudaSuccess)
@@ -137,15 +137,15 @@ bq_status quantize_tma(const uint16_t *W, int64_t N, int64_t K, uint8_t *packed,
   return launch_status();
 }
 
-template <int WT, int BITS>
+template <int WT, int BITS, int SCHEME>
 bq_status quantize_tiled(const uint16_t *W, int64_t N, int64_t K, int group, uint8_t *packed, float *scales,
                          uint8_t *zeros, cudaStream_t st) {
   switch (group) {
-    case 16: return quantize_tma<WT, BITS, 16>(W, N, K, packed, scales, zeros, st);
-    case 32: return quantize_tma<WT, BITS, 32>(W, N, K, packed, scales, zeros, st);
-    case 64: return quantize_tma<WT, BITS, 64>(W, N, K, packed, scales, zeros, st);
-    case 128: return quantize_tma<WT, BITS, 128>(W, N, K, packed, scales, zeros, st);
-    case 256: return quantize_tma<WT, BITS, 256>(W, N, K, packed, scales, zeros, st);
+    case 16: return quantize_tma<WT, BITS, 16, SCHEME>(W, N, K, packed, scales, zeros, st);
+    case 32: return quantize_tma<WT, BITS, 32, SCHEME>(W, N, K, packed, scales, zeros, st);
+    case 64: return quantize_tma<WT, BITS, 64, SCHEME>(W, N, K, packed, scales, zeros, st);
+    case 128: return quantize_tma<WT, BITS, 128, SCHEME>(W, N, K, packed, scales, zeros, st);
+    case 256: return quantize_tma<WT, BITS, 256, SCHEME>(W, N, K, packed, scales, zeros, st);
     default: return BQ_ERR_UNSUPPORTED;
   }
 }
@@ -440,6 +440,41 @@ bool linear_group_ok(int bits, int g) {
   return g == 32 || g == 64 || g == 128 || g == 256;
 }
 
+// bq_quantize / bq_quantize_symmetric: the same validation and layouts,
+// SCHEME 0 asymmetric MinMax, 1 symmetric abs-max.
+template <int SCHEME>
+bq_status quantize_any(const void *W, bq_dtype wtype, int64_t rows, int64_t cols, int bits, int group,
+                       bq_layout layout, void *packed, float *scales, uint8_t *zeros, void *stream) {
+  if (rows < 0 || cols < 0) return BQ_ERR_SHAPE;
+  if (!valid_bits(bits) || (wtype != BQ_F16 && wtype != BQ_BF16)) return BQ_ERR_UNSUPPORTED;
+  if (layout != BQ_LAYOUT_CANONICAL && layout != BQ_LAYOUT_INTERLEAVED) return BQ_ERR_UNSUPPORTED;
+  if (layout == BQ_LAYOUT_CANONICAL ? !canonical_group_ok(group) : !tiled_group_ok(group)) return BQ_ERR_UNSUPPORTED;
+  if (cols % group) return BQ_ERR_SHAPE;
+  if (layout == BQ_LAYOUT_CANONICAL) {
+    if ((cols * bits) % 32) return BQ_ERR_SHAPE;
+  } else {
+    const int64_t U = group > tile_width(bits) ? group : tile_width(bits);
+    if (rows % 16 || cols % U) return BQ_ERR_SHAPE;
+  }
+  if (rows == 0 || cols == 0) return BQ_OK;
+  if (!W || !packed || !scales || !zeros) return BQ_ERR_NULL;
+  if (!aligned(W, 16) || !aligned(packed, 16) || !aligned(scales, 4)) return BQ_ERR_ALIGN;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const uint16_t *w = reinterpret_cast<const uint16_t *>(W);
+  uint8_t *pk = reinterpret_cast<uint8_t *>(packed);
+  if (layout == BQ_LAYOUT_CANONICAL) {
+    const int64_t elems = rows * cols;
+    if (wtype == BQ_F16) return bits == 4 ? quantize_canonical<0, 4, SCHEME>(w, elems, group, pk, scales, zeros, st)
+                                          : quantize_canonical<0, 2, SCHEME>(w, elems, group, pk, scales, zeros, st);
+    return bits == 4 ? quantize_canonical<1, 4, SCHEME>(w, elems, group, pk, scales, zeros, st)
+                     : quantize_canonical<1, 2, SCHEME>(w, elems, group, pk, scales, zeros, st);
+  }
+  if (wtype == BQ_F16) return bits == 4 ? quantize_tiled<0, 4, SCHEME>(w, rows, cols, group, pk, scales, zeros, st)
+                                        : quantize_tiled<0, 2, SCHEME>(w, rows, cols, group, pk, scales, zeros, st);
+  return bits == 4 ? quantize_tiled<1, 4, SCHEME>(w, rows, cols, group, pk, scales, zeros, st)
+                   : quantize_tiled<1, 2, SCHEME>(w, rows, cols, group, pk, scales, zeros, st);
+}
+
 }  // namespace
 
 // ===========================================================================
@@ -495,34 +530,12 @@ bq_status bq_mixed_offsets(const uint8_t *bit_map, int64_t rows, int64_t cols, i
 
 bq_status bq_quantize(const void *W, bq_dtype wtype, int64_t rows, int64_t cols, int bits, int group,
                       bq_layout layout, void *packed, float *scales, uint8_t *zeros, void *stream) {
-  if (rows < 0 || cols < 0) return BQ_ERR_SHAPE;
-  if (!valid_bits(bits) || (wtype != BQ_F16 && wtype != BQ_BF16)) return BQ_ERR_UNSUPPORTED;
-  if (layout != BQ_LAYOUT_CANONICAL && layout != BQ_LAYOUT_INTERLEAVED) return BQ_ERR_UNSUPPORTED;
-  if (layout == BQ_LAYOUT_CANONICAL ? !canonical_group_ok(group) : !tiled_group_ok(group)) return BQ_ERR_UNSUPPORTED;
-  if (cols % group) return BQ_ERR_SHAPE;
-  if (layout == BQ_LAYOUT_CANONICAL) {
-    if ((cols * bits) % 32) return BQ_ERR_SHAPE;
-  } else {
-    const int64_t U = group > tile_width(bits) ? group : tile_width(bits);
-    if (rows % 16 || cols % U) return BQ_ERR_SHAPE;
-  }
-  if (rows == 0 || cols == 0) return BQ_OK;
-  if (!W || !packed || !scales || !zeros) return BQ_ERR_NULL;
-  if (!aligned(W, 16) || !aligned(packed, 16) || !aligned(scales, 4)) return BQ_ERR_ALIGN;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const uint16_t *w = reinterpret_cast<const uint16_t *>(W);
-  uint8_t *pk = reinterpret_cast<uint8_t *>(packed);
-  if (layout == BQ_LAYOUT_CANONICAL) {
-    const int64_t elems = rows * cols;
-    if (wtype == BQ_F16) return bits == 4 ? quantize_canonical<0, 4>(w, elems, group, pk, scales, zeros, st)
-                                          : quantize_canonical<0, 2>(w, elems, group, pk, scales, zeros, st);
-    return bits == 4 ? quantize_canonical<1, 4>(w, elems, group, pk, scales, zeros, st)
-                     : quantize_canonical<1, 2>(w, elems, group, pk, scales, zeros, st);
-  }
-  if (wtype == BQ_F16) return bits == 4 ? quantize_tiled<0, 4>(w, rows, cols, group, pk, scales, zeros, st)
-                                        : quantize_tiled<0, 2>(w, rows, cols, group, pk, scales, zeros, st);
-  return bits == 4 ? quantize_tiled<1, 4>(w, rows, cols, group, pk, scales, zeros, st)
-                   : quantize_tiled<1, 2>(w, rows, cols, group, pk, scales, zeros, st);
+  return quantize_any<0>(W, wtype, rows, cols, bits, group, layout, packed, scales, zeros, stream);
+}
+
+bq_status bq_quantize_symmetric(const void *W, bq_dtype wtype, int64_t rows, int64_t cols, int bits, int group,
+                                bq_layout layout, void *packed, float *scales, uint8_t *zeros, void *stream) {
+  return quantize_any<1>(W, wtype, rows, cols, bits, group, layout, packed, scales, zeros, stream);
 }
 
 bq_status bq_quantize_mixed(const void *W, bq_dtype wtype, int64_t rows, int64_t cols, const uint8_t *bit_map,

@@ -142,8 +142,40 @@ struct GroupParams {
   bool bad;      // non-finite input or overflowing scale
 };
 
+// Symmetric abs-max scheme ("大模型量化实战", section 2.3): s = max|x| /
+// (2^(b-1) - 1), zero point 0, codes stored offset by 2^(b-1) (z = 2^(b-1)),
+// so the same code rounding, storage and dequantization apply.  An all-zero
+// group stores s = 0 and every code equal to z.
 template <int QMAX>
+BQ_DEV GroupParams group_params_sym(float mn, float mx) {
+  constexpr int ZC = (QMAX + 1) / 2;
+  GroupParams p;
+  p.bad = !(fabsf(mn) <= 3.402823466e38f) || !(fabsf(mx) <= 3.402823466e38f);
+  const float amax = fmaxf(fabsf(mn), fabsf(mx));
+  const float s = __fdiv_rn(amax, (float)(ZC - 1));
+  p.bad |= !(s <= 3.402823466e38f);
+  p.z = ZC;
+  p.zc = ZC - kRoundMagicBits;
+  if (p.bad || s == 0.0f) {
+    p.s = 0.0f;
+    p.sd = 1.0f;
+    p.r = 1.0f;
+    p.fast = true;
+    p.clamp = true;
+    return p;
+  }
+  p.s = s;
+  p.sd = s;
+  p.fast = (s >= 8.67361738e-19f) && (s <= 1.15292150e18f);  // 2^-60 .. 2^60
+  p.r = __frcp_rn(s);
+  p.clamp = __float2int_rn(__fdiv_rn(amax, s)) + ZC > QMAX;
+  return p;
+}
+
+// SCHEME 0: asymmetric MinMax (below); 1: symmetric abs-max.
+template <int QMAX, int SCHEME = 0>
 BQ_DEV GroupParams group_params(float mn, float mx) {
+  if (SCHEME == 1) return group_params_sym<QMAX>(mn, mx);
   GroupParams p;
   p.bad = !(fabsf(mn) <= 3.402823466e38f) || !(fabsf(mx) <= 3.402823466e38f);
   float lo = fminf(mn, 0.0f);

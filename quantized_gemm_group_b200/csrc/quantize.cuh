@@ -33,7 +33,7 @@ namespace bq {
 
 // Quantize 8 consecutive weights held as 4 packed 16-bit pairs; the group
 // spans LANES = G/8 adjacent lanes.  Returns the 8 codes packed LSB-first.
-template <int WT, int BITS, int G>
+template <int WT, int BITS, int G, int SCHEME = 0>
 BQ_DEV uint32_t quant8_canonical(uint4 v, bool active, float *s_out, uint8_t *z_out, bool *bad) {
   using E = Elem<WT>;
   constexpr int LANES = G / 8;
@@ -49,7 +49,7 @@ BQ_DEV uint32_t quant8_canonical(uint4 v, bool active, float *s_out, uint8_t *z_
     mn = fmin_nan(mn, __shfl_xor_sync(0xffffffffu, mn, off));
     mx = fmax_nan(mx, __shfl_xor_sync(0xffffffffu, mx, off));
   }
-  GroupParams p = group_params<QMAX>(mn, mx);
+  GroupParams p = group_params<QMAX, SCHEME>(mn, mx);
   *s_out = p.s;
   *z_out = (uint8_t)p.z;
   *bad = p.bad;
@@ -64,7 +64,7 @@ BQ_DEV uint32_t quant8_canonical(uint4 v, bool active, float *s_out, uint8_t *z_
 
 // W viewed flat: element e of the matrix = W[e], groups of G start at
 // multiples of G, codes packed flat.
-template <int WT, int BITS, int G, int UNROLL>
+template <int WT, int BITS, int G, int UNROLL, int SCHEME = 0>
 __global__ void __launch_bounds__(256)
 quantize_canonical_kernel(const uint16_t *__restrict__ W, int64_t elems,
                           uint8_t *__restrict__ packed, float *__restrict__ scales,
@@ -90,7 +90,7 @@ quantize_canonical_kernel(const uint16_t *__restrict__ W, int64_t elems,
       float s;
       uint8_t z;
       bool bad;
-      uint32_t pk = quant8_canonical<WT, BITS, G>(v[u], act[u], &s, &z, &bad);
+      uint32_t pk = quant8_canonical<WT, BITS, G, SCHEME>(v[u], act[u], &s, &z, &bad);
       if (!act[u]) continue;
       bad_any |= bad;
       if (BITS == 4) {
@@ -176,7 +176,7 @@ BQ_DEV void codes_of_group(const UnitRegs<BITS, G> &u, int h, int gi, const Grou
 
 // Quantize one loaded unit: rows row0..row0+15, columns col0..col0+U-1 of an
 // N x K matrix; `packed`, `scales`, `zeros` are that matrix's own.
-template <int WT, int BITS, int G>
+template <int WT, int BITS, int G, int SCHEME = 0>
 BQ_DEV bool quantize_unit(const UnitRegs<BITS, G> &u, int64_t N, int64_t K, int64_t row0, int64_t col0,
                           uint8_t *__restrict__ packed, float *__restrict__ scales,
                           uint8_t *__restrict__ zeros, int lane) {
@@ -206,7 +206,7 @@ BQ_DEV bool quantize_unit(const UnitRegs<BITS, G> &u, int64_t N, int64_t K, int6
       mx = fmax_nan(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
       mn = fmin_nan(mn, __shfl_xor_sync(0xffffffffu, mn, 2));
       mx = fmax_nan(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      gp[h][gi] = group_params<QMAX>(mn, mx);
+      gp[h][gi] = group_params<QMAX, SCHEME>(mn, mx);
       bad_any |= gp[h][gi].bad;
     }
   }
@@ -277,7 +277,7 @@ BQ_DEV void load_unit_smem(UnitRegs<BITS, G> &u, uint32_t su, int t, int lane) {
   }
 }
 
-template <int WT, int BITS, int G>
+template <int WT, int BITS, int G, int SCHEME = 0>
 __global__ void __launch_bounds__(kQtThreads, 2)
 quantize_tma_kernel(const __grid_constant__ CUtensorMap wmap, int64_t N, int64_t K, int stages,
                     uint8_t *__restrict__ packed, float *__restrict__ scales, uint8_t *__restrict__ zeros) {
@@ -346,7 +346,7 @@ quantize_tma_kernel(const __grid_constant__ CUtensorMap wmap, int64_t N, int64_t
       load_unit_smem<BITS, G>(u, sbase + (uint32_t)slot * SU_BYTES, t, lane);
       __syncwarp();
       if (lane == 0) mbar_arrive(bars + 8u * (stages + slot));
-      bad |= quantize_unit<WT, BITS, G>(u, N, K, row0, col0, packed, scales, zeros, lane);
+      bad |= quantize_unit<WT, BITS, G, SCHEME>(u, N, K, row0, col0, packed, scales, zeros, lane);
     } else {
       __syncwarp();
       if (lane == 0) mbar_arrive(bars + 8u * (stages + slot));

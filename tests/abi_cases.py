@@ -50,6 +50,17 @@ def test_quantize_validation(L):
     assert q(L, layout=0, rows=3, cols=0, group=8, W=None) == bq.BQ_OK
 
 
+def test_quantize_symmetric_validation(L):
+    f = L.bq_quantize_symmetric
+    assert f(FAKE, bq.BQ_F16, 16, 128, 3, 128, 1, FAKE, FAKE, FAKE, None) == bq.BQ_ERR_UNSUPPORTED
+    assert f(FAKE, bq.BQ_F32, 16, 128, 4, 128, 1, FAKE, FAKE, FAKE, None) == bq.BQ_ERR_UNSUPPORTED
+    assert f(FAKE, bq.BQ_F16, 20, 128, 4, 128, 1, FAKE, FAKE, FAKE, None) == bq.BQ_ERR_SHAPE   # rows % 16
+    assert f(FAKE, bq.BQ_F16, 16, 192, 4, 128, 0, FAKE, FAKE, FAKE, None) == bq.BQ_ERR_SHAPE   # cols % group
+    assert f(None, bq.BQ_F16, 16, 128, 4, 128, 1, FAKE, FAKE, FAKE, None) == bq.BQ_ERR_NULL
+    assert f(FAKE_MIS, bq.BQ_F16, 16, 128, 4, 128, 1, FAKE, FAKE, FAKE, None) == bq.BQ_ERR_ALIGN
+    assert f(None, bq.BQ_F16, 0, 128, 4, 128, 1, None, None, None, None) == bq.BQ_OK
+
+
 def test_quantize_mixed_validation(L):
     f = L.bq_quantize_mixed
     assert f(FAKE, bq.BQ_F16, 200, 256, FAKE, 1, FAKE, FAKE, FAKE, None) == bq.BQ_ERR_SHAPE
