@@ -433,6 +433,31 @@ void bqo_linear_f64(const double *x, int64_t M, int64_t K,
     }
 }
 
+/* Input gradient of the same layer: the backward pass that training in the
+ * quantized weight space needs ([GB], the Bitorch Engine paragraph on
+ * gradients of low-bit tensors, and the Q-SFT paragraph).  With
+ * y = x . dequant(W)^T, the gradient with respect to x is dx = dy . dequant(W):
+ *   dx[m, k] = sum_n dy[m, n] * dequant(W)[n, k]   in fp64, n ascending,
+ * for input columns k in [k0, k1).  dy is [M, N] doubles, dx is [M, K]. */
+void bqo_linear_grad_input_f64(const double *dy, int64_t M, int64_t N,
+                               const uint8_t *codes, const float *scales, const uint8_t *zeros,
+                               int64_t K, int group, int64_t k0, int64_t k1,
+                               double *wcol /* scratch of N doubles */, double *dx)
+{
+    const int64_t G = K / group;
+    for (int64_t k = k0; k < k1 && k < K; ++k) {
+        const int64_t j = k / group;
+        for (int64_t n = 0; n < N; ++n)
+            wcol[n] = (double)((int)codes[n * K + k] - (int)zeros[n * G + j])
+                      * (double)scales[n * G + j];
+        for (int64_t m = 0; m < M; ++m) {
+            double acc = 0.0;
+            for (int64_t n = 0; n < N; ++n) acc += dy[m * N + n] * wcol[n];
+            dx[m * K + k] = acc;
+        }
+    }
+}
+
 /* Decode an fp16 (wtype 0) or bf16 (wtype 1) array to doubles. */
 void bqo_decode_f64(const uint16_t *src, int wtype, int64_t count, double *dst)
 {

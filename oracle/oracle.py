@@ -70,6 +70,8 @@ def lib():
             L.bqo_dequant_f32.restype = None
             L.bqo_linear_f64.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i64, i64, vp, vp]
             L.bqo_linear_f64.restype = None
+            L.bqo_linear_grad_input_f64.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i64, i64, vp, vp]
+            L.bqo_linear_grad_input_f64.restype = None
             L.bqo_decode_f64.argtypes = [vp, i32, i64, vp]
             L.bqo_decode_f64.restype = None
             L.bqo_meta_index.argtypes = [i32, i64, i64, i64, i64]
@@ -272,6 +274,29 @@ def linear_f64(x_f64: np.ndarray, codes, scales, zeros, group: int, threads: int
         with ThreadPoolExecutor(threads) as ex:
             list(ex.map(run, _row_chunks(N, threads)))
     return y
+
+
+def linear_grad_input_f64(dy_f64: np.ndarray, codes, scales, zeros, group: int, threads: int = 1) -> np.ndarray:
+    """dx = dy . dequant(W) in fp64 (n ascending).  dy_f64: [M, N] float64;
+    codes / scales / zeros as returned by quantize (row-major)."""
+    dy_f64 = np.ascontiguousarray(dy_f64, dtype=np.float64)
+    M, N = dy_f64.shape
+    K = codes.shape[1]
+    assert codes.shape[0] == N
+    dx = np.empty((M, K), dtype=np.float64)
+    L = lib()
+
+    def run(c):
+        scratch = np.empty(N, dtype=np.float64)
+        L.bqo_linear_grad_input_f64(_p(dy_f64), M, N, _p(codes), _p(scales), _p(zeros), K, group,
+                                    c[0], c[1], _p(scratch), _p(dx))
+
+    if threads <= 1:
+        run((0, K))
+    else:
+        with ThreadPoolExecutor(threads) as ex:
+            list(ex.map(run, _row_chunks(K, threads)))
+    return dx
 
 
 def to_bf16_bits(y: np.ndarray) -> np.ndarray:

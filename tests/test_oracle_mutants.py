@@ -37,6 +37,10 @@ MUTANTS = {
     "sym_no_offset": ("int q = (int)nearbyintf(x[i] / s) + z;", "int q = (int)nearbyintf(x[i] / s);"),
     "sym_round_half_away": ("int q = (int)nearbyintf(x[i] / s) + z;", "int q = (int)roundf(x[i] / s) + z;"),
     "sym_min_not_abs": ("float a = fabsf(x[i]);", "float a = x[i];"),
+    "grad_zero_sign": ("wcol[n] = (double)((int)codes[n * K + k] - (int)zeros[n * G + j])",
+                       "wcol[n] = (double)((int)codes[n * K + k] + (int)zeros[n * G + j])"),
+    "grad_dy_transposed": ("acc += dy[m * N + n] * wcol[n];", "acc += dy[n * M + m] * wcol[n];"),
+    "grad_group_of_column": ("const int64_t j = k / group;", "const int64_t j = (k / group) % (G > 1 ? G - 1 : 1);"),
 }
 
 # cheap pins first; each mutant only has to fail one of them
@@ -57,6 +61,8 @@ PINS = [
     (P.test_sym_worked_examples, {"name": "sym_int4_g8_worked.txt"}),
     (P.test_sym_worked_examples, {"name": "sym_int2_g8_worked.txt"}),
     (P.test_sym_page_scale_example, {}),
+    (P.test_grad_input_closed_form, {"bits": 4, "g": 128}),
+    (P.test_grad_input_adjoint, {"bits": 4, "g": 32}),
 ]
 
 

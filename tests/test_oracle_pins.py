@@ -10,6 +10,8 @@ and the mathematics fix, none of which re-types the oracle's own formulas.
   * packing: hand-derived positions, bijection, canonical word examples
   * element decoding against numpy / torch conversions
   * the linear layer against a closed form and an exactly-rounded sum
+  * its input gradient against a closed form, the adjoint identity with the
+    forward product, and one-hot rows of the dequantized matrix
 """
 from __future__ import annotations
 
@@ -415,6 +417,57 @@ def test_linear_exact_sum():
                      for k in range(K)]
             exact = math.fsum(terms)
             assert abs(y[m, n] - exact) <= 1e-13 * math.fsum(abs(t) for t in terms) + 1e-300
+
+
+@pytest.mark.parametrize("bits,g", [(4, 128), (2, 64)])
+def test_grad_input_closed_form(bits, g):
+    """dx = dy . W for a matrix the quantizer reproduces exactly, against
+    numpy's matmul."""
+    rng = np.random.default_rng(13 * bits)
+    N, K, M = 40, 256, 3
+    W, codes, scales, zeros = _representable_matrix(rng, N, K, g, bits)
+    c2, s2, z2 = O.quantize(W.astype(np.float16).view(np.uint16), "f16", bits, g)
+    assert (c2 == codes).all() and (s2 == scales).all() and (z2 == zeros).all()
+    dy = rng.normal(0, 1, (M, N)).astype(np.float16).astype(np.float64)
+    dx = O.linear_grad_input_f64(dy, c2, s2, z2, g, threads=2)
+    assert dx.shape == (M, K)
+    assert np.allclose(dx, dy @ W, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("bits,g", [(4, 32), (2, 64)])
+def test_grad_input_adjoint(bits, g):
+    """<dy, x . dequant(W)^T> = <dy . dequant(W), x>: the input gradient is the
+    adjoint of the forward product (pinned on its own above), here for
+    generic quantized weights."""
+    rng = np.random.default_rng(5 + bits)
+    N, K, M = 48, 256, 4
+    w = rng.normal(0, 0.02, (N, K)).astype(np.float16)
+    codes, scales, zeros = O.quantize(w.view(np.uint16), "f16", bits, g)
+    x = rng.normal(0, 1, (M, K))
+    dy = rng.normal(0, 1, (M, N))
+    y = O.linear_f64(x, codes, scales, zeros, g)
+    dx = O.linear_grad_input_f64(dy, codes, scales, zeros, g)
+    lhs = math.fsum((dy * y).ravel())
+    rhs = math.fsum((dx * x).ravel())
+    Wd = np.abs(O.dequant_f64(codes, scales, zeros, g))
+    bound = 1e-12 * float(np.sum(np.abs(dy) * (np.abs(x) @ Wd.T)))
+    assert abs(lhs - rhs) <= bound
+
+
+def test_grad_input_one_hot_rows():
+    """dy = one-hot (token m, channel n) gives dx[m] = row n of dequant(W) and
+    zero for every other token."""
+    rng = np.random.default_rng(17)
+    N, K, g = 20, 128, 32
+    w = rng.normal(0, 0.02, (N, K)).astype(np.float16)
+    codes, scales, zeros = O.quantize(w.view(np.uint16), "f16", 4, g)
+    Wd = O.dequant_f64(codes, scales, zeros, g)
+    for m, n in [(0, 0), (1, 7), (2, N - 1)]:
+        dy = np.zeros((3, N))
+        dy[m, n] = 1.0
+        dx = O.linear_grad_input_f64(dy, codes, scales, zeros, g)
+        assert (dx[m] == Wd[n]).all()
+        assert (np.delete(dx, m, axis=0) == 0).all()
 
 
 def test_mixed_offsets_hand_computed():
