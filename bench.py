@@ -343,6 +343,46 @@ def per_shape_numbers(stack, M, stream, reps=20):
     return res
 
 
+def grad_numbers(stack, Ms, hbm, reps=5):
+    """Input gradient dx = dy . dequant(W) (bq_linear_grad_input) over the
+    whole decode stack -- every fused projection of every layer, one CUDA
+    graph per token count; dy bf16 N(0,1).  GB/s of algorithmic bytes (packed
+    weights + metadata + dy + dx), CUDA-event median."""
+    res = {}
+    for M in Ms:
+        dys, dxs = {}, {}
+        for (_, _, N, K, _) in stack.fused:
+            if (N, K) not in dys:
+                dys[(N, K)] = synth.activations(M, N, seed=9, device="cuda")
+                dxs[(N, K)] = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+        s = torch.cuda.Stream()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g, stream=s):
+                for j, (_, _, N, K, _) in enumerate(stack.fused):
+                    pk, sc, ze = stack.fq[j]
+                    bq.bq_linear_grad_input(dys[(N, K)], pk, sc, ze, K, stack.bits, stack.group, out=dxs[(N, K)],
+                                            stream=s)
+        g.replay()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            g.replay()
+            b.record()
+            b.synchronize()
+            ts.append(a.elapsed_time(b) / 1e3)
+        t = statistics.median(ts)
+        byts = sum(linear_bytes(N, K, stack.bits, stack.group, M) for (_, _, N, K, _) in stack.fused)
+        res[str(M)] = {"ms": round(t * 1e3, 4), "GBps": round(byts / t / 1e9, 1),
+                       "frac_of_measured_hbm": round(byts / t / 1e9 / hbm, 4), "launches": len(stack.fused)}
+        del g
+    if bq.bq_device_status() != bq.BQ_OK:
+        raise RuntimeError("input-gradient kernel reported a device error")
+    return res
+
+
 def e2e_numbers(stack, Ms, steps, warmup, world):
     """Same metric through the C ABI with host buffers: every step copies all
     activations from pinned host memory to the device and all outputs back.
@@ -564,6 +604,8 @@ def run_gpu(args, world, rank, local):
                 "us_per_launch_avg": round(t_step / launches_per_step * 1e6, 3)}
 
     extra = {"per_M": per_m, "per_shape": shapes, "quantizer_stack": None}
+    if not args.no_grad:
+        extra["grad_input_stack"] = grad_numbers(stack, Ms, hbm)
     if not args.no_quant:
         extra["quantizer_8192x49152"] = quant_shape_numbers(hbm)
     if not args.no_gemm:
@@ -671,6 +713,7 @@ def main():
     ap.add_argument("--no-quant", action="store_true")
     ap.add_argument("--quick", action="store_true", help="skip the per-shape breakdown")
     ap.add_argument("--no-gemm", action="store_true", help="skip the prefill GEMM numbers")
+    ap.add_argument("--no-grad", action="store_true", help="skip the input-gradient (backward) numbers")
     ap.add_argument("--overlap", type=int, default=2, choices=[0, 1, 2],
                     help="bq_linear launch overlap: 0 plain, 1 programmatic dependent launch, "
                          "2 PDL + weight streaming before the wait (weights are static here)")

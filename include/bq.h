@@ -218,6 +218,30 @@ bq_status bq_linear(const void *x, bq_dtype xtype, int64_t M, int64_t K,
                     bq_layout layout, void *y, void *stream);
 
 /*
+ * bq_linear_grad_input: dx[M, K] = dy[M, N] . dequant(W), the gradient of
+ * bq_linear's output with respect to its input -- the backward pass of the
+ * layer when training in the quantized weight space (GreenBitAI article: the
+ * Bitorch Engine paragraph on gradients of low-bit tensors, and the Q-SFT
+ * paragraph).  W [N, K] is read in place; no dequantized copy is formed.
+ *   dy       [M, N] of dtype (BQ_BF16 or BQ_F16), 16-byte aligned
+ *   packed / scales / zeros: W from bq_quantize or bq_quantize_symmetric in
+ *            BQ_LAYOUT_INTERLEAVED, all three 16-byte aligned
+ *   bit_map  must be NULL (uniform width; BQ_ERR_UNSUPPORTED otherwise);
+ *            bits / group as in bq_linear
+ *   dx       [M, K] of dtype, written in full (N == 0: zeros, dy not read;
+ *            M == 0 or K == 0: nothing is done)
+ * dx[m, k] = sum_n dy[m, n] s[n, g] (q[n, k] - z[n, g]) on tensor cores with
+ * fp32 accumulation: (q - z) enters exactly, dy[m, n] s[n, g] is rounded once
+ * to tf32 (relative error at most 2^-11), dx is rounded once to dtype.  Runs
+ * in passes of at most 16 tokens, each reading W once.  Needs N % 16 == 0,
+ * K % 128 == 0 and K % group == 0.
+ */
+bq_status bq_linear_grad_input(const void *dy, bq_dtype dtype, int64_t M, int64_t N,
+                               const void *packed, const float *scales, const uint8_t *zeros,
+                               const uint8_t *bit_map, int bits, int group, int64_t K,
+                               bq_layout layout, void *dx, void *stream);
+
+/*
  * Options.
  *
  * BQ_OPT_LINEAR_OVERLAP (process-wide, default 0 or the value of the

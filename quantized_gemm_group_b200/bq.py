@@ -33,7 +33,7 @@ GROUP_OF_BITS = {4: 128, 2: 64}
 EXPORTS = (
     "bq_packed_bytes", "bq_group_count", "bq_mixed_offsets", "bq_quantize", "bq_quantize_symmetric",
     "bq_quantize_mixed",
-    "bq_dequantize", "bq_fake_quantize", "bq_linear", "bq_check_division", "bq_set_option", "bq_get_option", "bq_device_status",
+    "bq_dequantize", "bq_fake_quantize", "bq_linear", "bq_linear_grad_input", "bq_check_division", "bq_set_option", "bq_get_option", "bq_device_status",
     "bq_status_string", "bq_version",
 )
 BQ_OPT_LINEAR_OVERLAP = 0
@@ -77,6 +77,8 @@ def lib(path: str | None = None):
     L.bq_fake_quantize.restype = i32
     L.bq_linear.argtypes = [vp, i32, i64, i64, vp, vp, vp, vp, i32, i32, i64, i32, vp, vp]
     L.bq_linear.restype = i32
+    L.bq_linear_grad_input.argtypes = [vp, i32, i64, i64, vp, vp, vp, vp, i32, i32, i64, i32, vp, vp]
+    L.bq_linear_grad_input.restype = i32
     L.bq_check_division.argtypes = [ctypes.c_uint32, ctypes.c_uint32, i32, vp, vp]
     L.bq_check_division.restype = i32
     L.bq_set_option.argtypes = [i32, i32]
@@ -211,6 +213,19 @@ def bq_linear(x: torch.Tensor, packed, scales, zeros, N: int, bits: int = 4, gro
                          _ptr(bit_map_dev), bits, group, N, LAYOUTS[layout], _ptr(y), _stream(stream))
     _check("bq_linear", st)
     return y
+
+
+def bq_linear_grad_input(dy: torch.Tensor, packed, scales, zeros, K: int, bits: int = 4, group: int | None = None,
+                         layout: str = "interleaved", out=None, stream=None):
+    """dx [M, K] = dy [M, N] . dequant(W), dx in dy's dtype (the input
+    gradient of bq_linear)."""
+    group = group or GROUP_OF_BITS.get(bits, 0)
+    M, N = dy.shape
+    dx = out if out is not None else torch.empty((M, K), dtype=dy.dtype, device=dy.device)
+    st = lib().bq_linear_grad_input(_ptr(dy), DTYPE_CODE[dy.dtype], M, N, _ptr(packed), _ptr(scales), _ptr(zeros),
+                                    None, bits, group, K, LAYOUTS[layout], _ptr(dx), _stream(stream))
+    _check("bq_linear_grad_input", st)
+    return dx
 
 
 def bq_check_division(s_bits_begin: int, s_bits_end: int, refinements: int = 2, stream=None):

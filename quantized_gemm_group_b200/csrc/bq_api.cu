@@ -10,6 +10,7 @@
 #include "common.cuh"
 #include "dequant.cuh"
 #include "fakequant.cuh"
+#include "grad.cuh"
 #include "gemm.cuh"
 #include "gemv.cuh"
 #include "quantize.cuh"
@@ -358,6 +359,99 @@ bq_status gemv_dispatch(const uint16_t *x, int M, int64_t K, const uint8_t *pack
 }
 
 // ---------------------------------------------------------------------------
+// input gradient (M <= 16 per pass) geometry and dispatch
+// ---------------------------------------------------------------------------
+
+struct GradGeom {
+  int NB, d, stages;
+};
+
+// Cluster size d (CTAs splitting the rows of one 128-column slice, at most 8
+// and at most one per 128-row block): enough CTAs for two per SM; the ring
+// as deep as two CTAs per SM allow.
+GradGeom grad_geometry(int M, int64_t N, int64_t K, int gmax) {
+  GradGeom g;
+  g.NB = (M <= 8) ? 1 : 2;
+  const int64_t slices = K / kGradSlice, nbk = (N + 127) / 128;
+  int64_t d = (2 * sm_count()) / (slices > 0 ? slices : 1);
+  if (d > 8) d = 8;
+  if (d > nbk) d = nbk;
+  if (d < 1) d = 1;
+  g.d = (int)d;
+  g.stages = 2;
+  for (int s = kGradMaxStages; s >= 2; --s)
+    if (grad_smem_layout(M, 8 * g.NB, gmax, s, g.d).total <= kTwoCtaSmem) {
+      g.stages = s;
+      break;
+    }
+  return g;
+}
+
+template <int XT, int BITS, int G, int NB>
+bq_status launch_grad_t(const GradGeom &g, GradArgs a, cudaStream_t st) {
+  auto kern = grad_input_kernel<XT, BITS, G, NB>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem) != cudaSuccess)
+      return BQ_ERR_CUDA;
+    attr_set = true;
+  }
+  constexpr int gmax = (G <= kGradSlice) ? kGradSlice / G : 1;
+  a.stages = g.stages;
+  a.L = grad_smem_layout(a.M, 8 * NB, gmax, g.stages, g.d);
+  if (a.L.total > kMaxSmem) return BQ_ERR_SHAPE;
+  const int mode = overlap_mode();
+  a.prefetch_before_wait = (mode == 2) ? 1 : 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(a.K / kGradSlice), (unsigned)g.d, 1);
+  cfg.blockDim = dim3(32 * (kGradWarps + 1), 1, 1);
+  cfg.dynamicSmemBytes = (size_t)a.L.total;
+  cfg.stream = st;
+  cudaLaunchAttribute attrs[2];
+  int na = 0;
+  attrs[na].id = cudaLaunchAttributeClusterDimension;
+  attrs[na].val.clusterDim.x = 1;
+  attrs[na].val.clusterDim.y = (unsigned)g.d;
+  attrs[na].val.clusterDim.z = 1;
+  ++na;
+  if (mode >= 1) {
+    attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attrs[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  cfg.attrs = attrs;
+  cfg.numAttrs = na;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return BQ_ERR_CUDA;
+  }
+  return BQ_OK;
+}
+
+template <int XT>
+bq_status grad_dispatch(const uint16_t *dy, int M, int64_t N, const uint8_t *packed, const float *scales,
+                        const uint8_t *zeros, int bits, int group, int64_t K, uint16_t *dx, cudaStream_t st) {
+  GradArgs a = {};
+  a.dy = dy;
+  a.packed = packed;
+  a.scales = scales;
+  a.zeros = zeros;
+  a.dx = dx;
+  a.N = N;
+  a.K = K;
+  a.M = M;
+#define BQ_GD(B, G_)                                                                  \
+  if (bits == B && group == G_) {                                                     \
+    const GradGeom g = grad_geometry(M, N, K, (G_ <= kGradSlice) ? kGradSlice / G_ : 1); \
+    return g.NB == 1 ? launch_grad_t<XT, B, G_, 1>(g, a, st) : launch_grad_t<XT, B, G_, 2>(g, a, st); \
+  }
+  BQ_GD(4, 128) BQ_GD(2, 64) BQ_GD(4, 32) BQ_GD(4, 64) BQ_GD(4, 256) BQ_GD(2, 32) BQ_GD(2, 128) BQ_GD(2, 256)
+#undef BQ_GD
+  return BQ_ERR_UNSUPPORTED;
+}
+
+// ---------------------------------------------------------------------------
 // prefill GEMM (tcgen05)
 // ---------------------------------------------------------------------------
 
@@ -652,6 +746,36 @@ bq_status bq_linear(const void *x, bq_dtype xtype, int64_t M, int64_t K, const v
     bq_status s = (xtype == BQ_BF16)
                       ? gemv_dispatch<1>(xx + m0 * K, mb, K, pk, scales, zeros, bit_map, bits, group, N, yy + m0 * N, st)
                       : gemv_dispatch<0>(xx + m0 * K, mb, K, pk, scales, zeros, bit_map, bits, group, N, yy + m0 * N, st);
+    if (s != BQ_OK) return s;
+  }
+  return BQ_OK;
+}
+
+bq_status bq_linear_grad_input(const void *dy, bq_dtype dtype, int64_t M, int64_t N, const void *packed,
+                               const float *scales, const uint8_t *zeros, const uint8_t *bit_map, int bits,
+                               int group, int64_t K, bq_layout layout, void *dx, void *stream) {
+  if (M < 0 || K < 0 || N < 0) return BQ_ERR_SHAPE;
+  if (dtype != BQ_F16 && dtype != BQ_BF16) return BQ_ERR_UNSUPPORTED;
+  if (layout != BQ_LAYOUT_INTERLEAVED || bit_map) return BQ_ERR_UNSUPPORTED;
+  if (!valid_bits(bits) || !linear_group_ok(bits, group)) return BQ_ERR_UNSUPPORTED;
+  if (N % 16 || K % kGradSlice || K % group) return BQ_ERR_SHAPE;
+  if (M == 0 || K == 0) return BQ_OK;
+  if (!dx) return BQ_ERR_NULL;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (N == 0) {  // an empty sum: dy and W are not read
+    return cudaMemsetAsync(dx, 0, (size_t)(M * K * 2), st) == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+  }
+  if (!dy || !packed || !scales || !zeros) return BQ_ERR_NULL;
+  if (!aligned(dy, 16) || !aligned(dx, 16) || !aligned(packed, 16) || !aligned(scales, 16) || !aligned(zeros, 16))
+    return BQ_ERR_ALIGN;
+  const uint16_t *g = reinterpret_cast<const uint16_t *>(dy);
+  uint16_t *out = reinterpret_cast<uint16_t *>(dx);
+  const uint8_t *pk = reinterpret_cast<const uint8_t *>(packed);
+  for (int64_t m0 = 0; m0 < M; m0 += 16) {
+    const int mb = (int)((M - m0) < 16 ? (M - m0) : 16);
+    bq_status s = (dtype == BQ_BF16)
+                      ? grad_dispatch<1>(g + m0 * N, mb, N, pk, scales, zeros, bits, group, K, out + m0 * K, st)
+                      : grad_dispatch<0>(g + m0 * N, mb, N, pk, scales, zeros, bits, group, K, out + m0 * K, st);
     if (s != BQ_OK) return s;
   }
   return BQ_OK;

@@ -96,6 +96,31 @@ def test_linear_validation(L):
     assert lin(L, M=0, x=None, y=None) == bq.BQ_OK
 
 
+def grad(L, dy=FAKE, dt=bq.BQ_BF16, M=1, N=4096, pk=FAKE, sc=FAKE, ze=FAKE, bm=None, bits=4, group=128,
+         K=4096, layout=1, dx=FAKE):
+    return L.bq_linear_grad_input(dy, dt, M, N, pk, sc, ze, bm, bits, group, K, layout, dx, None)
+
+
+def test_linear_grad_input_validation(L):
+    assert grad(L, M=-1) == bq.BQ_ERR_SHAPE
+    assert grad(L, dt=bq.BQ_F32) == bq.BQ_ERR_UNSUPPORTED
+    assert grad(L, layout=0) == bq.BQ_ERR_UNSUPPORTED       # reads the interleaved layout
+    assert grad(L, bm=FAKE) == bq.BQ_ERR_UNSUPPORTED        # uniform width only
+    assert grad(L, bits=3) == bq.BQ_ERR_UNSUPPORTED
+    assert grad(L, group=16) == bq.BQ_ERR_UNSUPPORTED
+    assert grad(L, N=24) == bq.BQ_ERR_SHAPE                 # row tiles of 16
+    assert grad(L, K=4160) == bq.BQ_ERR_SHAPE               # 128-column slices
+    assert grad(L, K=4224, group=256) == bq.BQ_ERR_SHAPE    # K % group
+    assert grad(L, dy=None) == bq.BQ_ERR_NULL
+    assert grad(L, ze=None) == bq.BQ_ERR_NULL
+    assert grad(L, dx=None) == bq.BQ_ERR_NULL
+    assert grad(L, dy=FAKE_MIS) == bq.BQ_ERR_ALIGN
+    assert grad(L, dx=FAKE_MIS) == bq.BQ_ERR_ALIGN
+    assert grad(L, sc=FAKE_MIS) == bq.BQ_ERR_ALIGN
+    assert grad(L, M=0, dy=None, dx=None) == bq.BQ_OK
+    assert grad(L, K=0, dy=None, dx=None) == bq.BQ_OK
+
+
 def test_fake_quantize_validation(L):
     f = L.bq_fake_quantize
     assert f(FAKE, bq.BQ_F32, 16, 128, 4, 128, FAKE, bq.BQ_BF16, None) == bq.BQ_ERR_UNSUPPORTED  # W must be 16-bit
