@@ -22,17 +22,19 @@
 //  * The interleaved layout puts a row on lane / 4 and a column pair on
 //    lane % 4 -- the register order of the forward product, whose
 //    contraction runs over columns.  Here the contraction index must sit on
-//    lane % 4, so lane (g, t) reads the two 16-byte slots 4t + g/2 and
-//    4t + g/2 + 16 of the tile from shared memory: they hold rows t, t + 8
-//    and t + 4, t + 12 at columns g and g + 8 of every run.
+//    lane % 4, so lane (g, t) reads the two 16-byte slots 4t + g % 4 and
+//    4t + g % 4 + 16 of the tile from shared memory: they hold rows t, t + 8
+//    and t + 4, t + 12 at the columns 2 (g % 4) + 8 (g / 4) and the next one
+//    of every run (even column in the lower half-word, odd in the upper).
 //  * Operands: a code q at bit position p of a word becomes the fp32 value
 //    2^23 + q 2^p with one AND/OR against the exponent of 2^23, and one
 //    subtract of 2^23 + z 2^p leaves 2^p (q - z) exactly -- an exact tf32
-//    value.  Columns g + 8 sit 2 BITS bits above columns g and are shifted
-//    down first; the second 8-row half of a tile sits BITS bits above the
-//    first, a factor 2^BITS folded into the scale that multiplies its dy (an
-//    exact power-of-two scaling).  dy[m, n] s[n, g] is rounded once to tf32,
-//    the only rounding before the fp32 accumulation.
+//    value.  The second 8-row half of a tile sits BITS bits above the first,
+//    a factor 2^BITS folded into the scale that multiplies its dy; the high
+//    column pairs sit 2 BITS bits above the low ones, a factor taken off the
+//    lane's sums at the end (both exact power-of-two scalings).
+//    dy[m, n] s[n, g] is rounded once to tf32, the only rounding before the
+//    fp32 accumulation.
 //  * Warps' partial sums meet in shared memory (the idle ring) and are added
 //    in warp order; CTAs of a cluster split the rows and meet in distributed
 //    shared memory, added in rank order: deterministic, no global scratch.
@@ -185,7 +187,8 @@ BQ_DEV void grad_produce(const GradArgs &a, int64_t b0, int nblk, int64_t col0, 
 // 2 (w / 2) + 1 and runs 4 (w % 2) .. 4 (w % 2) + 3, so that a warp's partial
 // sums (16 tokens x 64 columns) stay in registers.  acc[run][token block]
 // [fragment] accumulates dx^T for the warp's runs: fragment q is column
-// 16 run + g + 8 (q / 2) and token 8 nb + 2t + (q % 2).
+// 16 run + 2 (g % 4) + 8 (g / 4) + q / 2 and token 8 nb + 2t + (q % 2), times
+// 2^(2 BITS (g / 4)) (undone when the sums leave the registers).
 template <int XT, int BITS, int G, int NB, int CW>
 BQ_DEV void grad_consume(const GradArgs &a, int w, int64_t b0, int nblk, uint32_t smem, uint32_t bars,
                          volatile int *abort, int lane, float (&acc)[8 / CW][NB][4]) {
@@ -201,9 +204,13 @@ BQ_DEV void grad_consume(const GradArgs &a, int w, int64_t b0, int nblk, uint32_
   const int S = a.stages;
   const int r_lo = (w % CW) * RW;                                 // the warp's first run
   const int rt0 = (w / CW) * CW;                                  // the warp's first row tile
-  const uint32_t slot1 = 16u * (uint32_t)(4 * t + (g >> 1));      // rows t, t + 8
+  // lane group g takes the column pair (2 (g % 4) + 8 (g / 4), + 1) of every
+  // run: both from the slots of column pair g % 4, whose slot index i =
+  // h + 2 (g / 4) puts them at bit BITS h + hpos of the lower (even column)
+  // and upper (odd column) half-word
+  const uint32_t slot1 = 16u * (uint32_t)(4 * t + (g & 3));       // rows t, t + 8
   const uint32_t slot2 = slot1 + 16u * 16u;                       // rows t + 4, t + 12
-  const uint32_t odd_shift = 16u * (uint32_t)(g & 1);             // odd columns: upper half-word
+  const uint32_t hpos = 2u * BITS * (uint32_t)(g >> 2);
   for (int i = 0; i < nblk; ++i) {
     const uint32_t st = smem + (uint32_t)((i % S) * a.L.sb);
     const uint32_t full = bars + 8u * (i % S), empty = bars + 8u * (S + i % S);
@@ -235,7 +242,7 @@ BQ_DEV void grad_consume(const GradArgs &a, int w, int64_t b0, int nblk, uint32_
             asm volatile("ld.shared.u8 %0, [%1];" : "=r"(z) : "r"(st + a.L.z_off + gi * rows + nl));
             // the second half tile's codes sit BITS bits higher: scale its dy' down by 2^BITS
             const float sh = h ? s * (1.0f / (float)(1 << BITS)) : s;
-            cz[h][aa] = __fmaf_rn((float)z, (float)(1u << (BITS * h)), 8388608.0f);  // 2^23 + z 2^(BITS h)
+            cz[h][aa] = __uint_as_float(kMagic | (z << (BITS * h + hpos)));  // 2^23 + z 2^(BITS h + hpos)
 #pragma unroll
             for (int nb = 0; nb < NB; ++nb) {
               const int m = g + 8 * nb;
@@ -254,21 +261,23 @@ BQ_DEV void grad_consume(const GradArgs &a, int w, int64_t b0, int nblk, uint32_
           const int rs = r_lo + rl;      // run within the slice
           const int ct = rs / RPT;       // column tile
           const int wj = (BITS == 4) ? (rs % RPT) : (rs % RPT) / 2;
-          // r_lo is even, so the parity of rs is that of rl
-          const uint32_t shift = odd_shift + ((BITS == 2) ? 8u * (uint32_t)(rl & 1) : 0u);
           const uint32_t tb = st + (uint32_t)((ct * R + rt) * 512 + wj * 4);
-          // lo: columns g of rows (t, t + 8) / (t + 4, t + 12) at bit BITS h;
-          // hi: columns g + 8, 2 BITS bits higher, shifted down to the same place
-          const uint32_t w1 = lds_u32(tb + slot1) >> shift, w1h = w1 >> (2 * BITS);
-          const uint32_t w2 = lds_u32(tb + slot2) >> shift, w2h = w2 >> (2 * BITS);
+          uint32_t w1 = lds_u32(tb + slot1), w2 = lds_u32(tb + slot2);
+          // 2 bits: the word's second run sits 8 bits higher (r_lo is even, so
+          // the parity of rs is that of rl)
+          if (BITS == 2 && (rl & 1)) {
+            w1 >>= 8;
+            w2 >>= 8;
+          }
+          const uint32_t w1o = w1 >> 16, w2o = w2 >> 16;  // odd columns
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const uint32_t mask = QM << (BITS * h);
+            const uint32_t mask = QM << (BITS * h + hpos);
             uint32_t av[4];
             av[0] = __float_as_uint(__fsub_rn(__uint_as_float(and_or(w1, mask, kMagic)), cz[h][0]));
-            av[1] = __float_as_uint(__fsub_rn(__uint_as_float(and_or(w1h, mask, kMagic)), cz[h][0]));
+            av[1] = __float_as_uint(__fsub_rn(__uint_as_float(and_or(w1o, mask, kMagic)), cz[h][0]));
             av[2] = __float_as_uint(__fsub_rn(__uint_as_float(and_or(w2, mask, kMagic)), cz[h][1]));
-            av[3] = __float_as_uint(__fsub_rn(__uint_as_float(and_or(w2h, mask, kMagic)), cz[h][1]));
+            av[3] = __float_as_uint(__fsub_rn(__uint_as_float(and_or(w2o, mask, kMagic)), cz[h][1]));
 #pragma unroll
             for (int nb = 0; nb < NB; ++nb) mma_tf32(acc[rl][nb], av, bp[nb][h][0], bp[nb][h][1]);
           }
@@ -335,7 +344,8 @@ __global__ void __launch_bounds__(32 * (kGradWarps + 1), 2) grad_input_kernel(co
   float *red = reinterpret_cast<float *>(smem_raw);
   if (warp < kGradWarps) {
     const int g = lane >> 2, t = lane & 3;
-    const int rgw = warp / CW, c0 = 16 * (warp % CW) * RW;
+    const int rgw = warp / CW, c0 = 16 * (warp % CW) * RW + 2 * (g & 3) + 8 * (g >> 2);
+    const float unscale = (g >> 2) ? 1.0f / (float)(1 << (2 * BITS)) : 1.0f;  // exact
 #pragma unroll
     for (int r = 0; r < RW; ++r)
 #pragma unroll
@@ -343,8 +353,8 @@ __global__ void __launch_bounds__(32 * (kGradWarps + 1), 2) grad_input_kernel(co
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int m = 8 * nb + 2 * t + (q & 1);
-          const int col = c0 + 16 * r + g + 8 * (q >> 1);
-          red[(rgw * TOK + m) * kGradRedStride + col] = acc[r][nb][q];
+          const int col = c0 + 16 * r + (q >> 1);
+          red[(rgw * TOK + m) * kGradRedStride + col] = acc[r][nb][q] * unscale;
         }
   }
   __syncthreads();
