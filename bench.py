@@ -54,9 +54,10 @@ FALLBACK_BF16_TFLOPS = 1590.0
 M_SET = (1, 4, 16)
 # DRAM bytes (read + write) per algorithmic byte of the decode kernel, from
 # the ncu capture of gemv_kernel on gate_up 28672x4096 INT4 at M = 1
-# (profiles/gemv_kernel_gate_up_28672x4096_int4.md: 63.654 MB for 63.37 MB);
-# the kernel reads every weight byte once, so traffic scales with the bytes.
-GEMV_DRAM_PER_ALGO_BYTE = 63.654 / 63.37
+# (profiles/gemv_kernel_gate_up_28672x4096_int4.md: 63,492,608 DRAM bytes read
+# and written for 63,373,312 algorithmic bytes); the kernel reads every weight
+# byte once, so traffic scales with the bytes.
+GEMV_DRAM_PER_ALGO_BYTE = 63492608 / 63373312
 METRIC = "W4/W2 dequant-GEMV weight GB/s (M<=16) & GEMM TFLOP/s (M>=2048) vs roofline"
 
 

@@ -381,6 +381,9 @@ gemv_kernel(const GemvArgs a) {
   float *part = reinterpret_cast<float *>(smem_raw + a.L.part_off);
 
   pdl_launch_dependents();
+  // every CTA of the cluster must have started before any writes into
+  // another's shared memory (the matching wait precedes those writes)
+  if (SK > 1) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 
   // the zero chunk read by padding tokens
   if (threadIdx.x == 0) *reinterpret_cast<uint4 *>(smem_raw + a.L.zero_off) = make_uint4(0, 0, 0, 0);
@@ -467,6 +470,7 @@ gemv_kernel(const GemvArgs a) {
   // rank order.  No remote access follows the barrier.
   const int E = TOK * ROWS;
   const int per = (E + SK - 1) / SK;
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
   if (warp < R) {
     const int r = lane >> 2, c = lane & 3;
 #pragma unroll
