@@ -384,6 +384,66 @@ def grad_numbers(stack, Ms, hbm, reps=5):
     return res
 
 
+def mixed_numbers(layers, Ms, hbm, reps=5):
+    """Decode stack with per-128-row-block widths (4 bits -> group 128, 2 bits
+    -> group 64): Layer-mix (one width per layer, 8 of 32 layers at 4 bits)
+    and Channel-mix (25% of the blocks of every matrix at 4 bits).  Weights
+    fp16 N(0, 0.02), one fused matrix per linear; x bf16 N(0, 1).  GB/s of
+    algorithmic bytes (each block's codes + metadata, x, y) over one CUDA
+    graph per token count, CUDA-event median."""
+    res = {}
+    lmap = synth.layer_mix_map(layers)
+    for kind in ("layer_mix", "channel_mix"):
+        mods = []
+        for i, (l, _, N, K, _) in enumerate(fused_shapes(layers)):
+            W = synth.normal((N, K), 0.02, seed=500000 + i, dtype="f16", device="cuda")
+            if kind == "layer_mix":
+                bmap = [lmap[l]] * (N // 128)
+            else:
+                bmap = synth.channel_mix_map(N, seed=600000 + i).tolist()
+            pk, sc, ze, bm = bq.bq_quantize_mixed(W, bmap, "interleaved")
+            del W
+            wb = sum(weight_bytes(128, K, b, 128 if b == 4 else 64) for b in bmap)
+            mods.append((N, K, pk, sc, ze, bm, wb, 128 * K * bmap.count(4)))
+        torch.cuda.synchronize()
+        if bq.bq_device_status() != bq.BQ_OK:
+            raise RuntimeError("mixed quantizer reported a device error")
+        weights4 = sum(m[7] for m in mods)
+        weights = sum(N * K for (N, K, *_rest) in mods)
+        per_m = {}
+        for M in Ms:
+            xs = {K: synth.activations(M, K, seed=7, device="cuda") for K in {m[1] for m in mods}}
+            ys = {N: torch.empty((M, N), dtype=torch.bfloat16, device="cuda") for N in {m[0] for m in mods}}
+            s = torch.cuda.Stream()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(s):
+                with torch.cuda.graph(g, stream=s):
+                    for (N, K, pk, sc, ze, bm, *_rest) in mods:
+                        bq.bq_linear(xs[K], pk, sc, ze, N, bit_map_dev=bm, out=ys[N], stream=s)
+            g.replay()
+            torch.cuda.synchronize()
+            ts = []
+            for _ in range(reps):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                g.replay()
+                b.record()
+                b.synchronize()
+                ts.append(a.elapsed_time(b) / 1e3)
+            t = statistics.median(ts)
+            byts = sum(m[6] + 2 * M * m[1] + 2 * M * m[0] for m in mods)
+            per_m[str(M)] = {"ms": round(t * 1e3, 4), "GBps": round(byts / t / 1e9, 1),
+                             "frac_of_measured_hbm": round(byts / t / 1e9 / hbm, 4)}
+            del g
+        if bq.bq_device_status() != bq.BQ_OK:
+            raise RuntimeError("mixed linear reported a device error")
+        res[kind] = {"bpw_codes": round((4 * weights4 + 2 * (weights - weights4)) / weights, 4), "launches": len(mods),
+                     "per_M": per_m}
+        del mods
+        torch.cuda.empty_cache()
+    return res
+
+
 def e2e_numbers(stack, Ms, steps, warmup, world):
     """Same metric through the C ABI with host buffers: every step copies all
     activations from pinned host memory to the device and all outputs back.
@@ -607,6 +667,8 @@ def run_gpu(args, world, rank, local):
     extra = {"per_M": per_m, "per_shape": shapes, "quantizer_stack": None}
     if not args.no_grad:
         extra["grad_input_stack"] = grad_numbers(stack, Ms, hbm)
+    if args.mixed:
+        extra["mixed_stack"] = mixed_numbers(args.layers, Ms, hbm)
     if not args.no_quant:
         extra["quantizer_8192x49152"] = quant_shape_numbers(hbm)
     if not args.no_gemm:
@@ -715,6 +777,8 @@ def main():
     ap.add_argument("--quick", action="store_true", help="skip the per-shape breakdown")
     ap.add_argument("--no-gemm", action="store_true", help="skip the prefill GEMM numbers")
     ap.add_argument("--no-grad", action="store_true", help="skip the input-gradient (backward) numbers")
+    ap.add_argument("--mixed", action="store_true",
+                    help="also time the Layer-mix / Channel-mix decode stacks (extra weights; off by default)")
     ap.add_argument("--overlap", type=int, default=2, choices=[0, 1, 2],
                     help="bq_linear launch overlap: 0 plain, 1 programmatic dependent launch, "
                          "2 PDL + weight streaming before the wait (weights are static here)")
