@@ -21,6 +21,8 @@
  * Low-bit Large Language Models", section 6.2 weight-only: dequantize, then a
  * 16-bit matmul; "大模型量化实战" section 3.3: dequantize and multiply in one
  * fused kernel).  No dequantized weight is ever written by the linear layer.
+ * Its input gradient dx = dy . dequant(W) (bq_linear_grad_input) reads the
+ * same packed weights in place.
  *
  * Conventions for every entry point
  * ---------------------------------
@@ -33,7 +35,9 @@
  *    stream).  Work is enqueued asynchronously; argument errors are returned
  *    synchronously before anything is enqueued.
  *  - Pointers to W, x, y, packed codes and dequantized output must be 16-byte
- *    aligned; scales and zeros 4-byte and 1-byte aligned.
+ *    aligned; scales and zeros 4-byte and 1-byte aligned, except for
+ *    bq_linear and bq_linear_grad_input, which read them with bulk copies
+ *    and need 16-byte alignment.
  *  - Conditions only the device can see (a non-finite weight, a wait that
  *    gave up) set a device status word; read it with bq_device_status().
  *  - On a CUDA launch failure the entry point returns BQ_ERR_CUDA.
