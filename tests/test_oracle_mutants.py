@@ -41,6 +41,16 @@ MUTANTS = {
                        "wcol[n] = (double)((int)codes[n * K + k] + (int)zeros[n * G + j])"),
     "grad_dy_transposed": ("acc += dy[m * N + n] * wcol[n];", "acc += dy[n * M + m] * wcol[n];"),
     "grad_group_of_column": ("const int64_t j = k / group;", "const int64_t j = (k / group) % (G > 1 ? G - 1 : 1);"),
+    "dequant32_zero_sign": ("float d = (float)((int)codes[n * cols + k] - (int)zeros[n * G + j]);",
+                            "float d = (float)((int)codes[n * cols + k] + (int)zeros[n * G + j]);"),
+    "dequant32_scale_transposed": ("out[n * cols + k] = d * scales[n * G + j];",
+                                   "out[n * cols + k] = d * scales[j * rows + n];"),
+    "dequant32_group_of_column": ("            int64_t j = k / group;\n            float d",
+                                  "            int64_t j = k % G;\n            float d"),
+    "dequant64_zero_sign": ("out[n * cols + k] = (double)((int)codes[n * cols + k] - (int)zeros[n * G + j])",
+                            "out[n * cols + k] = (double)((int)codes[n * cols + k] + (int)zeros[n * G + j])"),
+    "dequant64_scale_transposed": ("                                * (double)scales[n * G + j];\n        }\n}",
+                                   "                                * (double)scales[j * rows + n];\n        }\n}"),
 }
 
 # cheap pins first; each mutant only has to fail one of them
@@ -50,6 +60,8 @@ PINS = [
     (P.test_worked_examples, {"name": "int4_clamp_worked.txt"}),
     (P.test_worked_examples, {"name": "int4_zero_tie_worked.txt"}),
     (P.test_page_scale_example, {}),
+    (P.test_dequant_two_rows_two_groups, {}),
+    (P.test_mixed_dequant_and_linear_tiled, {}),
     (P.test_constant_groups, {}),
     (P.test_interleaved_positions_hand_derived, {}),
     (P.test_meta_positions_hand_derived, {}),

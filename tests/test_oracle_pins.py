@@ -98,10 +98,62 @@ def test_worked_examples(name):
     assert q.tolist() == [int(v) for v in g["q"]]
     deq = (q.astype(np.float64) - z) * s
     assert deq.tolist() == [float(v) for v in g["dequant"]]
+    # the oracle's own dequantization functions reproduce the hand-worked values
+    c1, s1, z1 = q.reshape(1, -1).astype(np.uint8), np.array([[s]], np.float32), np.array([[z]], np.uint8)
+    assert O.dequant_f32(c1, s1, z1, x.size)[0].tolist() == [float(v) for v in g["dequant"]]
+    assert O.dequant_f64(c1, s1, z1, x.size)[0].tolist() == [float(v) for v in g["dequant"]]
     for key in ("canonical_word32", "canonical_word16"):
         if key in g:
             packed = O.pack(q.reshape(1, -1), bits, "canonical")
             assert int.from_bytes(packed.tobytes(), "little") == int(g[key][0], 16)
+
+
+def _f16_bits(vals) -> np.ndarray:
+    return np.array(vals, dtype=np.float16).view(np.uint16)
+
+
+def test_dequant_two_rows_two_groups():
+    """Hand-worked matrix with a different scale per (row, group): the
+    oracle's quantizer gives the hand-worked codes, scales and zeros, and both
+    dequantization functions return (q - z) * s of the right row and group."""
+    g = read_golden("int4_2x2_groups_worked.txt")
+    bits, group = int(g["bits"][0]), int(g["group"][0])
+    x = np.stack([np.array([float(v) for v in g[f"x{r}"]]) for r in (0, 1)])
+    codes, scales, zeros = O.quantize(_f16_bits(x), "f16", bits, group)
+    assert codes.tolist() == [[int(v) for v in g[f"q{r}"]] for r in (0, 1)]
+    assert scales.reshape(-1).tolist() == [float(v) for v in g["scales"]]
+    assert zeros.reshape(-1).tolist() == [int(v) for v in g["zeros"]]
+    want = [[float(v) for v in g[f"dequant{r}"]] for r in (0, 1)]
+    assert O.dequant_f32(codes, scales, zeros, group).tolist() == want
+    assert O.dequant_f64(codes, scales, zeros, group).tolist() == want
+
+
+def test_mixed_dequant_and_linear_tiled():
+    """Mixed widths through the oracle's block-by-block path: a 4-bit block
+    (group 128) whose rows repeat the 8-element 4-bit worked example and a
+    2-bit block (group 64) whose rows repeat the 2-bit one.  Repeating a
+    group's vector keeps its min and max, so every group has the worked
+    example's scale, zero point and codes; the dequantized matrix is the
+    worked dequantization repeated, and a one-hot x selects its columns."""
+    g4, g2 = read_golden("int4_g8_worked.txt"), read_golden("int2_g8_worked.txt")
+    K = 128
+    rows4 = np.tile(np.array([float(v) for v in g4["x"]]), K // 8)
+    rows2 = np.tile(np.array([float(v) for v in g2["x"]]), K // 8)
+    W = np.concatenate([np.tile(rows4, (128, 1)), np.tile(rows2, (128, 1))])
+    bit_map = [4, 2]
+    _, _, _, blocks = O.quantize_mixed(_f16_bits(W), "f16", bit_map, "interleaved")
+    want = np.concatenate([np.tile(np.array([float(v) for v in g4["dequant"]]), (128, K // 8)),
+                           np.tile(np.array([float(v) for v in g2["dequant"]]), (128, K // 8))])
+    got = np.concatenate([O.dequant_f32(c, s, z, O.GROUP_OF_BITS[b]) for (c, s, z), b in zip(blocks, bit_map)])
+    assert (got == want).all()
+    for (c, s, z), b in zip(blocks, bit_map):
+        assert (s == float((g4 if b == 4 else g2)["s"][0])).all()
+        assert (z == int((g4 if b == 4 else g2)["z"][0])).all()
+    for k in (0, 5, 7, 64, 127):
+        x = np.zeros((1, K))
+        x[0, k] = 1.0
+        y = O.linear_mixed_f64(x, blocks, bit_map)
+        assert (y[0] == want[:, k]).all()
 
 
 def test_page_scale_example():
