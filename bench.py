@@ -53,11 +53,11 @@ FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 M_SET = (1, 4, 16)
 # DRAM bytes (read + write) per algorithmic byte of the decode kernel, from
-# the ncu capture of gemv_kernel on gate_up 28672x4096 INT4 at M = 1
-# (profiles/gemv_kernel_gate_up_28672x4096_int4.md: 63,492,608 DRAM bytes read
-# and written for 63,373,312 algorithmic bytes); the kernel reads every weight
-# byte once, so traffic scales with the bytes.
-GEMV_DRAM_PER_ALGO_BYTE = 63492608 / 63373312
+# one ncu capture of gemv_kernel on the gate_up 28672x4096 INT4 linear at
+# M = 1 (63,343,360 bytes read + 155,392 written for 63,373,312 algorithmic
+# bytes); the kernel reads every weight byte once, so traffic scales with
+# the bytes.
+GEMV_DRAM_PER_ALGO_BYTE = (63343360 + 155392) / 63373312
 METRIC = "W4/W2 dequant-GEMV weight GB/s (M<=16) & GEMM TFLOP/s (M>=2048) vs roofline"
 
 
@@ -444,6 +444,24 @@ def mixed_numbers(layers, Ms, hbm, reps=5):
     return res
 
 
+def stack_per_m(stack, Ms, hbm, steps, world):
+    """Decode numbers of one stack: one CUDA graph per token count."""
+    xs = {M: [synth.activations(M, K, seed=20000 * M + i, device="cuda")
+              for i, (_, _, N, K, _) in enumerate(stack.fused)] for M in Ms}
+    ys = {M: [torch.empty((M, N), dtype=torch.bfloat16, device="cuda") for (_, _, N, K, _) in stack.fused]
+          for M in Ms}
+    stream = torch.cuda.Stream()
+    per_m = {}
+    for M in Ms:
+        g = stack.make_graph((M,), xs, ys, stream)
+        tm = max_over_ranks(time_graph(g, steps, 1, stream, world) / steps, world)
+        bm = stack.step_bytes((M,))
+        per_m[str(M)] = {"ms": round(tm * 1e3, 4), "GBps": round(bm / tm / 1e9, 1),
+                         "frac_of_measured_hbm": round(bm / tm / 1e9 / hbm, 4), "tokens_per_s": round(M / tm, 1)}
+        del g
+    return per_m
+
+
 def e2e_numbers(stack, Ms, steps, warmup, world):
     """Same metric through the C ABI with host buffers: every step copies all
     activations from pinned host memory to the device and all outputs back.
@@ -560,6 +578,7 @@ def quant_shape_numbers(hbm, reps=10):
 
 
 GEMM_SHAPES = ((14336, 4096), (4096, 14336), (49152, 8192), (8192, 49152))
+GEMM_M = (2048, 4096, 8192)
 
 
 def gemm_numbers(Ms, bf16, bf16_sus, reps=10):
@@ -594,6 +613,34 @@ def gemm_numbers(Ms, bf16, bf16_sus, reps=10):
             del pk, sc, ze
         del W
         torch.cuda.empty_cache()
+    # Channel-mix (25% of the 128-row blocks at 4 bits, the rest at 2 bits)
+    # through the same tensor-core path
+    N, K = 14336, 4096
+    W = synth.normal((N, K), 0.015, seed=N + K, dtype="f16", device="cuda")
+    bmap = synth.channel_mix_map(N, seed=77).tolist()
+    pk, sc, ze, bm = bq.bq_quantize_mixed(W, bmap, "interleaved")
+    del W
+    for M in Ms[:1]:
+        x = synth.activations(M, K, seed=M, device="cuda")
+        y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        for _ in range(3):
+            bq.bq_linear(x, pk, sc, ze, N, bit_map_dev=bm, out=y)
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            bq.bq_linear(x, pk, sc, ze, N, bit_map_dev=bm, out=y)
+            b.record()
+            b.synchronize()
+            ts.append(a.elapsed_time(b) / 1e3)
+        t = statistics.median(ts)
+        tf = 2.0 * M * N * K / t / 1e12
+        res[f"{N}x{K} Channel-mix 2.5 bpw M{M}"] = {"us": round(t * 1e6, 1), "TFLOPs": round(tf, 1),
+                                                    "frac_of_measured_bf16_burst": round(tf / bf16, 4),
+                                                    "frac_of_measured_bf16_sustained": round(tf / bf16_sus, 4)}
+    del pk, sc, ze, bm
+    torch.cuda.empty_cache()
     if bq.bq_device_status() != bq.BQ_OK:
         raise RuntimeError("GEMM reported a device error")
     return res
@@ -647,6 +694,7 @@ def run_gpu(args, world, rank, local):
     step_bytes = stack.step_bytes(Ms)
     value = world * step_bytes / t_step / 1e9
     launches_per_step = len(Ms) * len(stack.fused)
+    packed_gb = sum(weight_bytes(N, K, bits, group) for (_, _, N, K, _) in stack.fused) / 1e9
 
     # end to end through the C ABI with host buffers
     t_e2e, h2d, d2h = e2e_numbers(stack, Ms, max(1, args.steps // 2), 2, world)
@@ -656,39 +704,54 @@ def run_gpu(args, world, rank, local):
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                 "frac": round(achieved / hbm, 4),
                 "traffic": round(GEMV_DRAM_PER_ALGO_BYTE * step_bytes / launches_per_step) if bits == 4 else None,
-                "traffic_note": "bytes per launch: ncu DRAM bytes per algorithmic byte of the committed capture "
-                                "x this step's algorithmic bytes per launch",
+                "traffic_note": "bytes per launch: ncu DRAM bytes per algorithmic byte of one capture of the "
+                                "kernel (gate_up 28672x4096, M = 1) x this step's algorithmic bytes per launch",
                 "kernel": "gemv_kernel (decode dequant-GEMV, mma.sync bf16)",
                 "peak_kind": peak_kind + " (copy burst)",
                 "frac_of_nominal_8TBps": round(achieved / 8000.0, 4),
                 "bytes_per_launch_avg": round(step_bytes / launches_per_step),
                 "us_per_launch_avg": round(t_step / launches_per_step * 1e6, 3)}
 
+    def quant_summary(qz):
+        return {"weights": qz["weights"], "ms": round(qz["seconds"] * 1e3, 3),
+                "weights_per_s": round(qz["weights_per_s"], 1), "GBps": round(qz["GBps"], 1),
+                "frac_of_measured_hbm": round(qz["GBps"] / hbm, 4), "launches": qz["launches"]}
+
     extra = {"per_M": per_m, "per_shape": shapes, "quantizer_stack": None}
     if not args.no_grad:
         extra["grad_input_stack"] = grad_numbers(stack, Ms, hbm)
-    if args.mixed:
-        extra["mixed_stack"] = mixed_numbers(args.layers, Ms, hbm)
+    if not args.no_gemm:
+        del g
+    if stack.quant:
+        extra["quantizer_stack"] = quant_summary(stack.quant)
+    if not args.no_other_width:
+        # the other width's stack (INT2 g64 on heavy-tailed weights with
+        # outlier columns, or INT4 g128 on N(0, 0.02)): quantizer over all of
+        # its weights and the decode numbers per token count
+        obits = 2 if bits == 4 else 4
+        del stack
+        torch.cuda.empty_cache()
+        other = Stack(args.layers, obits, 128 if obits == 4 else 64, seed_offset=rank * 100000 + 7,
+                      dist_kind="t4" if obits == 2 else "normal", quant_time=not args.no_quant)
+        extra[f"int{obits}_stack"] = {
+            "weights": "fp16 Student-t4 std 0.02 + 0.1% x10 outlier cols" if obits == 2 else "fp16 N(0,0.02)",
+            "group": 128 if obits == 4 else 64, "per_M": stack_per_m(other, Ms, hbm, max(2, args.steps), world),
+            "quantizer_stack": quant_summary(other.quant) if other.quant else None}
+        del other
+        torch.cuda.empty_cache()
+    if not args.no_mixed:
+        extra["mixed_stack"] = mixed_numbers(args.layers, (1, 16), hbm)
     if not args.no_quant:
         extra["quantizer_8192x49152"] = quant_shape_numbers(hbm)
     if not args.no_gemm:
-        del g
-        extra["prefill_gemm"] = gemm_numbers((2048, 8192) if not args.quick else (2048,), bf16,
-                                             bf16_sus or bf16)
-    if stack.quant:
-        qz = stack.quant
-        extra["quantizer_stack"] = {"weights": qz["weights"], "ms": round(qz["seconds"] * 1e3, 3),
-                                    "weights_per_s": round(qz["weights_per_s"], 1),
-                                    "GBps": round(qz["GBps"], 1), "frac_of_measured_hbm": round(qz["GBps"] / hbm, 4),
-                                    "launches": qz["launches"]}
+        extra["prefill_gemm"] = gemm_numbers(GEMM_M if not args.quick else (2048,), bf16, bf16_sus or bf16)
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(t_step * 1e3, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": f"bf16 x int{bits} -> fp32 acc", "data": "synthetic",
         "config": {**workload_config(args),
                    "weights": "fp16 N(0,0.02)" if bits == 4 else "fp16 Student-t4 std 0.02 + 0.1% x10 outlier cols",
-                   "activations": "bf16 N(0,1)", "l2": "inputs larger than L2 (packed stack %.2f GB)" %
-                   (sum(weight_bytes(N, K, bits, group) for (_, _, N, K, _) in stack.fused) / 1e9),
+                   "activations": "bf16 N(0,1)", "l2": "inputs larger than L2 (packed stack %.2f GB)" % packed_gb,
                    "graph": "one CUDA graph per step", "overlap": args.overlap,
                    "parallelism": f"replicas x{world} (independent batches)"},
         "roofline": roofline,
@@ -730,11 +793,50 @@ def oracle_sample(threads: int, layers_sample: int = 1, Ms=M_SET, bits=4):
 
 
 def cpu_baseline(args):
+    """The CPU oracle as it stands, on bounded samples of the workloads (about
+    half a minute of CPU work): the decode linear on all host cores (the
+    headline `value`) and on one core, the quantizer on all cores and on one,
+    and the prefill product on 256 tokens, extrapolated per multiply-add to
+    the largest prefill shape."""
+    from oracle import oracle as O  # test infrastructure, CPU baseline only
     threads = os.cpu_count() or 1
-    gbps, secs, byts = oracle_sample(threads, args.oracle_layers, bits=args.bits)
+    bits, group = args.bits, (128 if args.bits == 4 else 64)
+    gbps, secs, byts = oracle_sample(threads, args.oracle_layers, bits=bits)
+    gbps1, secs1, byts1 = oracle_sample(1, 1, Ms=(1,), bits=bits)
+    # quantizer: the first layer's seven weight matrices
+    Ws = [synth.normal((N, K), 0.02, synth.weight_seed(0, m), "f16", "cpu")
+          for m, (_, N, K) in enumerate(synth.LLAMA3_8B_LINEARS)]
+    nweights = sum(W.numel() for W in Ws)
+    t0 = time.perf_counter()
+    for W in Ws:
+        O.quantize(synth.bits16(W), "f16", bits, group, threads=threads)
+    tq = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    O.quantize(synth.bits16(Ws[0]), "f16", bits, group, threads=1)
+    tq1 = time.perf_counter() - t0
+    qbytes = nweights * 2 + sum(weight_bytes(W.shape[0], W.shape[1], bits, group) for W in Ws)
+    # prefill: 256 tokens against a 4096x4096 weight, per multiply-add
+    W = Ws[0]
+    c, sc, ze = O.quantize(synth.bits16(W), "f16", bits, group, threads=threads)
+    x = O.decode_f64(synth.bits16(synth.activations(256, W.shape[1], seed=3, device="cpu")), "bf16")
+    t0 = time.perf_counter()
+    O.linear_f64(x, c, sc, ze, group, threads=threads)
+    tg = time.perf_counter() - t0
+    macs_per_s = 256 * W.shape[0] * W.shape[1] / tg
+    big = 8192 * 49152 * 8192
     return {"value": round(gbps, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
             "sample": f"first {args.oracle_layers} layer(s) x 4 linears (qkv, o, gate_up, down) x M in {{1,4,16}} "
-                      f"({byts / 1e6:.1f} MB of weight traffic, {secs:.1f} s); fp64 linear over dequantized weights"}
+                      f"({byts / 1e6:.1f} MB of weight traffic, {secs:.1f} s); fp64 linear over dequantized weights",
+            "single_core": {"value": round(gbps1, 4), "unit": "GB/s", "cores": 1,
+                            "sample": f"first layer's 4 linears at M = 1 ({byts1 / 1e6:.1f} MB, {secs1:.1f} s)"},
+            "quantizer": {"weights_per_s": round(nweights / tq, 1), "GBps": round(qbytes / tq / 1e9, 4),
+                          "cores": threads, "weights_per_s_single_core": round(Ws[0].numel() / tq1, 1),
+                          "sample": f"first layer's 7 weight matrices ({nweights / 1e6:.0f} M weights, {tq:.1f} s; "
+                                    f"one core: q 4096x4096, {tq1:.1f} s), INT{bits} g{group}"},
+            "prefill_extrapolated": {"TFLOPs": round(2 * macs_per_s / 1e12, 6), "cores": threads,
+                                     "seconds_8192x49152_M8192": round(big / macs_per_s, 1),
+                                     "sample": f"256 tokens x 4096x4096 fp64 ({tg:.1f} s), extrapolated per "
+                                               "multiply-add (not measured at full size)"}}
 
 
 def run_reference(args, world, rank):
@@ -771,14 +873,15 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--bits", type=int, default=4, choices=[2, 4])
     ap.add_argument("--layers", type=int, default=synth.LLAMA3_8B_LAYERS)
-    ap.add_argument("--oracle-layers", type=int, default=1)
+    ap.add_argument("--oracle-layers", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-quant", action="store_true")
     ap.add_argument("--quick", action="store_true", help="skip the per-shape breakdown")
     ap.add_argument("--no-gemm", action="store_true", help="skip the prefill GEMM numbers")
     ap.add_argument("--no-grad", action="store_true", help="skip the input-gradient (backward) numbers")
-    ap.add_argument("--mixed", action="store_true",
-                    help="also time the Layer-mix / Channel-mix decode stacks (extra weights; off by default)")
+    ap.add_argument("--no-mixed", action="store_true", help="skip the Layer-mix / Channel-mix decode stacks")
+    ap.add_argument("--no-other-width", action="store_true",
+                    help="skip the second stack at the other width (INT2 g64 when timing INT4)")
     ap.add_argument("--overlap", type=int, default=2, choices=[0, 1, 2],
                     help="bq_linear launch overlap: 0 plain, 1 programmatic dependent launch, "
                          "2 PDL + weight streaming before the wait (weights are static here)")

@@ -41,6 +41,8 @@
  *  - Conditions only the device can see (a non-finite weight, a wait that
  *    gave up) set a device status word; read it with bq_device_status().
  *  - On a CUDA launch failure the entry point returns BQ_ERR_CUDA.
+ *  - Every entry point may be called from several host threads and for
+ *    several devices in one process (kernel attributes are set per device).
  */
 #ifndef BQ_H
 #define BQ_H
@@ -286,6 +288,17 @@ bq_status bq_device_status(void *stream);
  */
 bq_status bq_check_division(uint32_t s_bits_begin, uint32_t s_bits_end, int refinements,
                             unsigned long long *result, void *stream);
+
+/*
+ * bq_selftest_bounded_wait: diagnostic of the failure path of the kernels'
+ * bounded waits.  Launches one small kernel on `stream` that waits, with the
+ * same routine every kernel of the library uses, on a shared-memory barrier
+ * phase that nothing ever completes, giving up after `limit` polls (1 to
+ * 2^20).  The kernel then records BQ_ERR_TIMEOUT in the device status word
+ * and returns normally; nothing hangs and the context stays usable.  The next
+ * bq_device_status() returns BQ_ERR_TIMEOUT (and clears it).
+ */
+bq_status bq_selftest_bounded_wait(uint32_t limit, void *stream);
 
 /* Human-readable name of a status code (static string). */
 const char *bq_status_string(bq_status status);

@@ -33,7 +33,8 @@ GROUP_OF_BITS = {4: 128, 2: 64}
 EXPORTS = (
     "bq_packed_bytes", "bq_group_count", "bq_mixed_offsets", "bq_quantize", "bq_quantize_symmetric",
     "bq_quantize_mixed",
-    "bq_dequantize", "bq_fake_quantize", "bq_linear", "bq_linear_grad_input", "bq_check_division", "bq_set_option", "bq_get_option", "bq_device_status",
+    "bq_dequantize", "bq_fake_quantize", "bq_linear", "bq_linear_grad_input", "bq_check_division",
+    "bq_selftest_bounded_wait", "bq_set_option", "bq_get_option", "bq_device_status",
     "bq_status_string", "bq_version",
 )
 BQ_OPT_LINEAR_OVERLAP = 0
@@ -81,6 +82,8 @@ def lib(path: str | None = None):
     L.bq_linear_grad_input.restype = i32
     L.bq_check_division.argtypes = [ctypes.c_uint32, ctypes.c_uint32, i32, vp, vp]
     L.bq_check_division.restype = i32
+    L.bq_selftest_bounded_wait.argtypes = [ctypes.c_uint32, vp]
+    L.bq_selftest_bounded_wait.restype = i32
     L.bq_set_option.argtypes = [i32, i32]
     L.bq_set_option.restype = i32
     L.bq_get_option.argtypes = [i32]
@@ -235,6 +238,10 @@ def bq_check_division(s_bits_begin: int, s_bits_end: int, refinements: int = 2, 
                                                         _stream(stream)))
     torch.cuda.synchronize()
     return tuple(int(v) for v in res.cpu())
+
+
+def bq_selftest_bounded_wait(limit: int, stream=None):
+    _check("bq_selftest_bounded_wait", lib().bq_selftest_bounded_wait(limit, _stream(stream)))
 
 
 def bq_set_option(option: int, value: int):

@@ -1,6 +1,7 @@
 // bq_api.cu -- C ABI of the quantizer / weight-only linear library (see
 // include/bq.h for the contract of every entry point).  Host-side argument
 // validation, launch geometry and dispatch onto the sm_100a kernels.
+#include <atomic>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -36,6 +37,28 @@ int sm_count() {
 }
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+constexpr int kMaxDevices = 64;
+
+// cudaFuncAttributeMaxDynamicSharedMemorySize is a per-device setting of a
+// kernel: it is set on each device the first time the kernel needs more than
+// the default there (one record per kernel -- the template argument is the
+// kernel itself, not its type, which instantiations share -- and device; two
+// threads racing only set it twice).
+template <auto Kern>
+bool ensure_smem(int bytes) {
+  static std::atomic<int> set_to[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (dev >= 0 && dev < kMaxDevices && set_to[dev].load(std::memory_order_acquire) >= bytes) return true;
+  if (cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+  if (dev >= 0 && dev < kMaxDevices) {
+    int cur = set_to[dev].load(std::memory_order_relaxed);
+    while (cur < bytes && !set_to[dev].compare_exchange_weak(cur, bytes, std::memory_order_acq_rel)) {
+    }
+  }
+  return true;
+}
 
 bq_status launch_status() {
   cudaError_t e = cudaGetLastError();
@@ -119,12 +142,7 @@ bq_status quantize_tma(const uint16_t *W, int64_t N, int64_t K, uint8_t *packed,
   constexpr int SU = (U / 64) * 8192;
   constexpr int kBudget = 113 * 1024;
   auto kern = quantize_tma_kernel<WT, BITS, G, SCHEME>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kBudget) != cudaSuccess)
-      return BQ_ERR_CUDA;
-    attr_set = true;
-  }
+  if (!ensure_smem<quantize_tma_kernel<WT, BITS, G, SCHEME>>(kBudget)) return BQ_ERR_CUDA;
   int stages = (kBudget - 1024 - 16) / (SU + 16);
   if (stages > 8) stages = 8;
   if (stages < 2) return BQ_ERR_UNSUPPORTED;
@@ -219,15 +237,18 @@ bq_status dequant_mixed(const uint8_t *packed, const float *scales, const uint8_
 // 0: plain launches; 1: programmatic dependent launch (the kernel waits for
 // the previous one before reading anything); 2: as 1, and weights may be
 // streamed before that wait (the caller guarantees the preceding kernel does
-// not write them).
-int g_overlap_mode = -1;
+// not write them).  -1: not read from the environment yet.
+std::atomic<int> g_overlap_mode{-1};
 
 int overlap_mode() {
-  if (g_overlap_mode < 0) {
+  int m = g_overlap_mode.load(std::memory_order_relaxed);
+  if (m < 0) {
     const char *e = getenv("BQ_OVERLAP");
-    g_overlap_mode = (e && (e[0] == '1' || e[0] == '2')) ? e[0] - '0' : 0;
+    const int v = (e && (e[0] == '1' || e[0] == '2')) ? e[0] - '0' : 0;
+    g_overlap_mode.compare_exchange_strong(m, v);
+    m = g_overlap_mode.load(std::memory_order_relaxed);
   }
-  return g_overlap_mode;
+  return m;
 }
 
 struct GemvGeom {
@@ -285,12 +306,7 @@ GemvGeom gemv_geometry(int M, int64_t N, int64_t K, int SC, int G_min) {
 template <int XT, int BITS, int G, int NB, bool MIXED>
 bq_status launch_gemv_t(const GemvGeom &g, GemvArgs a, int G_min, cudaStream_t st) {
   auto kern = gemv_kernel<XT, BITS, G, NB, MIXED>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem) != cudaSuccess)
-      return BQ_ERR_CUDA;
-    attr_set = true;
-  }
+  if (!ensure_smem<gemv_kernel<XT, BITS, G, NB, MIXED>>(kMaxSmem)) return BQ_ERR_CUDA;
   a.stages = g.stages;
   a.KC = g.KC;
   a.L = gemv_smem_layout(a.M, 8 * NB, g.KC, (int)(g.KC / G_min), g.stages);
@@ -390,12 +406,7 @@ GradGeom grad_geometry(int M, int64_t N, int64_t K, int gmax) {
 template <int XT, int BITS, int G, int NB>
 bq_status launch_grad_t(const GradGeom &g, GradArgs a, cudaStream_t st) {
   auto kern = grad_input_kernel<XT, BITS, G, NB>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem) != cudaSuccess)
-      return BQ_ERR_CUDA;
-    attr_set = true;
-  }
+  if (!ensure_smem<grad_input_kernel<XT, BITS, G, NB>>(kMaxSmem)) return BQ_ERR_CUDA;
   constexpr int gmax = (G <= kGradSlice) ? kGradSlice / G : 1;
   a.stages = g.stages;
   a.L = grad_smem_layout(a.M, 8 * NB, gmax, g.stages, g.d);
@@ -465,20 +476,20 @@ bool make_x_map(CUtensorMap *map, const uint16_t *x, int64_t M, int64_t K, int x
   return make_map_2d(map, x, M, K, xt == 1, 64, kGemmTokTile);
 }
 
-template <int XT, int BITS, int G>
+template <int XT, int BITS, int G, bool MIXED = false>
 bq_status launch_gemm_t(const uint16_t *x, int64_t M, int64_t K, const GemmArgs &a, cudaStream_t st) {
-  auto kern = gemm_kernel<XT, BITS, G>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GemmSmem::total) != cudaSuccess)
-      return BQ_ERR_CUDA;
-    // the warpgroups' setmaxnreg shares must fit in the registers the block
-    // is launched with, or the raising warpgroups would wait forever
+  auto kern = gemm_kernel<XT, BITS, G, MIXED>;
+  // the warpgroups' setmaxnreg shares must fit in the registers the block is
+  // launched with, or the raising warpgroups would wait forever (a property
+  // of the compiled kernel, checked once per process)
+  static std::atomic<int> regs_ok{0};  // 0 unknown, 1 ok, -1 too few
+  if (regs_ok.load(std::memory_order_acquire) == 0) {
     cudaFuncAttributes fa;
     if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return BQ_ERR_CUDA;
-    if ((int64_t)fa.numRegs * kGemmThreads < (int64_t)kGemmRegsNeeded) return BQ_ERR_UNSUPPORTED;
-    attr_set = true;
+    regs_ok.store((int64_t)fa.numRegs * kGemmThreads >= (int64_t)kGemmRegsNeeded ? 1 : -1, std::memory_order_release);
   }
+  if (regs_ok.load(std::memory_order_acquire) < 0) return BQ_ERR_UNSUPPORTED;
+  if (!ensure_smem<gemm_kernel<XT, BITS, G, MIXED>>(GemmSmem::total)) return BQ_ERR_CUDA;
   CUtensorMap map;
   if (!make_x_map(&map, x, M, K, XT)) return BQ_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
@@ -503,25 +514,27 @@ bq_status launch_gemm_t(const uint16_t *x, int64_t M, int64_t K, const GemmArgs 
   return BQ_OK;
 }
 
-// Uniform width, N a multiple of 128 (whole blocks), groups a multiple of 64
-// columns, at least kGemmMinTokens tokens.
+// N a multiple of 128 (whole blocks), groups a multiple of 64 columns (a
+// width map's groups 128 and 64 are), at least kGemmMinTokens tokens.
 bool gemm_eligible(int64_t M, int64_t N, const uint8_t *bit_map, int group) {
-  return M >= kGemmMinTokens && !bit_map && N % kGemmRowTile == 0 && group % kGemmChunk == 0 &&
+  return M >= kGemmMinTokens && N % kGemmRowTile == 0 && (bit_map || group % kGemmChunk == 0) &&
          M <= 65535LL * kGemmTokTile;
 }
 
 template <int XT>
 bq_status gemm_dispatch(const uint16_t *x, int64_t M, int64_t K, const uint8_t *packed, const float *scales,
-                        const uint8_t *zeros, int bits, int group, int64_t N, uint16_t *y, cudaStream_t st) {
+                        const uint8_t *zeros, const uint8_t *bit_map, int bits, int group, int64_t N, uint16_t *y,
+                        cudaStream_t st) {
   GemmArgs a = {};
   a.packed = packed;
   a.scales = scales;
   a.zeros = zeros;
-  a.bit_map = nullptr;
+  a.bit_map = bit_map;
   a.y = y;
   a.M = M;
   a.K = K;
   a.N = N;
+  if (bit_map) return launch_gemm_t<XT, 4, 128, true>(x, M, K, a, st);
 #define BQ_GM(B, G_) \
   if (bits == B && group == G_) return launch_gemm_t<XT, B, G_>(x, M, K, a, st);
   BQ_GM(4, 128) BQ_GM(2, 64) BQ_GM(4, 64) BQ_GM(4, 256) BQ_GM(2, 128) BQ_GM(2, 256)
@@ -738,8 +751,8 @@ bq_status bq_linear(const void *x, bq_dtype xtype, int64_t M, int64_t K, const v
   uint16_t *yy = reinterpret_cast<uint16_t *>(y);
   const uint8_t *pk = reinterpret_cast<const uint8_t *>(packed);
   if (gemm_eligible(M, N, bit_map, group))
-    return (xtype == BQ_BF16) ? gemm_dispatch<1>(xx, M, K, pk, scales, zeros, bits, group, N, yy, st)
-                              : gemm_dispatch<0>(xx, M, K, pk, scales, zeros, bits, group, N, yy, st);
+    return (xtype == BQ_BF16) ? gemm_dispatch<1>(xx, M, K, pk, scales, zeros, bit_map, bits, group, N, yy, st)
+                              : gemm_dispatch<0>(xx, M, K, pk, scales, zeros, bit_map, bits, group, N, yy, st);
   // Otherwise token blocks of at most 16 go through the decode kernel.
   for (int64_t m0 = 0; m0 < M; m0 += 16) {
     const int mb = (int)((M - m0) < 16 ? (M - m0) : 16);
@@ -793,10 +806,16 @@ bq_status bq_check_division(uint32_t s_bits_begin, uint32_t s_bits_end, int refi
   return launch_status();
 }
 
+bq_status bq_selftest_bounded_wait(uint32_t limit, void *stream) {
+  if (limit < 1 || limit > (1u << 20)) return BQ_ERR_UNSUPPORTED;
+  bounded_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit);
+  return launch_status();
+}
+
 bq_status bq_set_option(int option, int value) {
   if (option == BQ_OPT_LINEAR_OVERLAP) {
     if (value < 0 || value > 2) return BQ_ERR_UNSUPPORTED;
-    g_overlap_mode = value;
+    g_overlap_mode.store(value);
     return BQ_OK;
   }
   return BQ_ERR_UNSUPPORTED;

@@ -295,9 +295,15 @@ BQ_DEV void gemm_dequant(const GemmArgs &a, int d, int lane, uint32_t sbase, con
   int st = 0, ph = 0, ws = 0, wph = 0;
   for (int ci = 0; ci < nchunks; ++ci) {
     const int cin = ci % GG::CPS;  // chunk inside the code stage
-    if (cin == 0 && !mbar_wait(B.w_full + 8u * ws, wph)) { *abort = 1; bq_flag(BQ_FLAG_TIMEOUT); break; }
-    if (ci >= kGemmAStages && !mbar_wait(B.a_empty + 8u * st, ph ^ 1)) { *abort = 1; bq_flag(BQ_FLAG_TIMEOUT); break; }
-    if (*abort) break;
+    // every wait is voted on, so the whole warp leaves together
+    if (!__all_sync(0xffffffffu, (*abort == 0) && (cin != 0 || mbar_wait(B.w_full + 8u * ws, wph)) &&
+                                     (ci < kGemmAStages || mbar_wait(B.a_empty + 8u * st, ph ^ 1)))) {
+      if (lane == 0) {
+        *abort = 1;
+        bq_flag(BQ_FLAG_TIMEOUT);
+      }
+      break;
+    }
     const uint32_t wst = sbase + GemmSmem::w_off + ws * GemmSmem::W_BYTES;
     const uint32_t zst = sbase + GemmSmem::z_off + ws * GemmSmem::Z_BYTES;
     const uint32_t ast = sbase + GemmSmem::a_off + st * GemmSmem::A_BYTES;
@@ -422,7 +428,13 @@ BQ_DEV void gemm_epilogue(const GemmArgs &a, const float *sc, int e, int warp, i
     const int buf = g & 1;
     const float s = s_next;
     if (g + 1 < ngroups) s_next = __ldg(sc + (int64_t)(g + 1) * 128 + rloc);
-    if (!mbar_wait(d_full + 8u * buf, (g >> 1) & 1)) { *abort = 1; bq_flag(BQ_FLAG_TIMEOUT); ok = false; break; }
+    // tcgen05.ld below is warp-collective: the whole warp leaves together
+    if (!__all_sync(0xffffffffu, mbar_wait(d_full + 8u * buf, (g >> 1) & 1))) {
+      *abort = 1;
+      bq_flag(BQ_FLAG_TIMEOUT);
+      ok = false;
+      break;
+    }
     tc_fence_after();
     const float2 s2 = make_float2(s, s);
 #pragma unroll
@@ -451,9 +463,32 @@ BQ_DEV void gemm_epilogue(const GemmArgs &a, const float *sc, int e, int warp, i
   }
 }
 
-// grid = (N / 128 weight blocks, ceil(M / 256) token tiles); 768 threads;
-// one CTA per SM (shared memory), all 512 TMEM columns.
+// The roles of one CTA for a block of width BITS, group G.
 template <int XT, int BITS, int G>
+BQ_DEV void gemm_roles(const GemmArgs &a, const CUtensorMap *xmap, const uint8_t *pk, const float *sc,
+                       const uint8_t *ze, int warp, int lane, uint32_t tmem, uint32_t sbase, const GemmBars &B,
+                       volatile int *abort, int64_t row0, int tok0) {
+  if (warp < kGemmWarpDeq0) {
+    setmaxnreg_dec<kGemmRegsCtl>();
+    if (warp == kGemmWarpProd && lane == 0) gemm_produce<BITS, G>(a, xmap, pk, ze, tok0, sbase, B, abort);
+    if ((warp == kGemmWarpMma || warp == kGemmWarpMma + 1) && lane == 0)
+      gemm_mma<XT, BITS, G>(a, warp - kGemmWarpMma, tmem, sbase, B, abort);
+  } else if (warp < kGemmWarpEpi0) {
+    setmaxnreg_dec<kGemmRegsDeq>();
+    gemm_dequant<XT, BITS, G>(a, warp - kGemmWarpDeq0, lane, sbase, B, abort);
+  } else {
+    setmaxnreg_inc<kGemmRegsEpi>();
+    gemm_epilogue<XT, BITS, G>(a, sc, warp - kGemmWarpEpi0, warp, lane, tmem, sbase, B, abort, row0, tok0);
+  }
+}
+
+// grid = (N / 128 weight blocks, ceil(M / 256) token tiles); 768 threads;
+// one CTA per SM (shared memory), all 512 TMEM columns.  MIXED: a width map
+// (Layer-mix / Channel-mix) gives each 128-row block 4 bits (group 128) or 2
+// bits (group 64); the CTA's block has one width, so it runs that width's
+// roles, its codes and metadata found by running sums over the map (a block
+// of b bits holds 16 K b code bytes and 128 K / group metadata entries).
+template <int XT, int BITS, int G, bool MIXED>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap xmap, const GemmArgs a) {
   extern __shared__ __align__(1024) unsigned char gsm_raw[];
@@ -467,6 +502,38 @@ gemm_kernel(const __grid_constant__ CUtensorMap xmap, const GemmArgs a) {
   const int64_t blk = blockIdx.x;
   const int64_t row0 = blk * kGemmRowTile;
   const int tok0 = blockIdx.y * kGemmTokTile;
+
+  // width of this block and where its codes / metadata start
+  int bits = BITS;
+  const uint8_t *pk;
+  const float *sc;
+  const uint8_t *ze;
+  if (!MIXED) {
+    pk = a.packed + blk * kGemmRowTile * a.K * BITS / 8;
+    sc = a.scales + blk * kGemmRowTile * (a.K / G);
+    ze = a.zeros + blk * kGemmRowTile * (a.K / G);
+  } else {
+    // every warp sums the map over the blocks before this one (shuffles)
+    int64_t sb = 0, sg = 0;
+    for (int64_t jb = lane; jb < blk; jb += 32) {
+      const int b = a.bit_map[jb];
+      sb += b;
+      sg += (b == 4) ? 1 : 2;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      sb += __shfl_xor_sync(0xffffffffu, sb, off);
+      sg += __shfl_xor_sync(0xffffffffu, sg, off);
+    }
+    bits = a.bit_map[blk];
+    pk = a.packed + sb * 16 * a.K;
+    sc = a.scales + sg * a.K;
+    ze = a.zeros + sg * a.K;
+    if (bits != 4 && bits != 2) {  // the whole CTA leaves before allocating anything
+      if (threadIdx.x == 0) bq_flag(BQ_FLAG_BADMAP);
+      return;
+    }
+  }
 
   const GemmBars B(sbase + GemmSmem::bar_off);
   if (threadIdx.x == 0) {
@@ -498,23 +565,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap xmap, const GemmArgs a) {
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const uint8_t *pk = a.packed + blk * kGemmRowTile * a.K * BITS / 8;
-  const float *sc = a.scales + blk * kGemmRowTile * (a.K / G);
-  const uint8_t *ze = a.zeros + blk * kGemmRowTile * (a.K / G);
-
   pdl_wait();
-  if (warp < kGemmWarpDeq0) {
-    setmaxnreg_dec<kGemmRegsCtl>();
-    if (warp == kGemmWarpProd && lane == 0) gemm_produce<BITS, G>(a, &xmap, pk, ze, tok0, sbase, B, abort);
-    if ((warp == kGemmWarpMma || warp == kGemmWarpMma + 1) && lane == 0)
-      gemm_mma<XT, BITS, G>(a, warp - kGemmWarpMma, tmem, sbase, B, abort);
-  } else if (warp < kGemmWarpEpi0) {
-    setmaxnreg_dec<kGemmRegsDeq>();
-    gemm_dequant<XT, BITS, G>(a, warp - kGemmWarpDeq0, lane, sbase, B, abort);
-  } else {
-    setmaxnreg_inc<kGemmRegsEpi>();
-    gemm_epilogue<XT, BITS, G>(a, sc, warp - kGemmWarpEpi0, warp, lane, tmem, sbase, B, abort, row0, tok0);
-  }
+  if (!MIXED || bits == BITS) gemm_roles<XT, BITS, G>(a, &xmap, pk, sc, ze, warp, lane, tmem, sbase, B, abort, row0, tok0);
+  else gemm_roles<XT, 2, 64>(a, &xmap, pk, sc, ze, warp, lane, tmem, sbase, B, abort, row0, tok0);
 
   // everything issued by this CTA has finished before the tensor memory goes
   tc_fence_before();

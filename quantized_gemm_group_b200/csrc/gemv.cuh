@@ -257,9 +257,13 @@ BQ_DEV void gemv_consume(const GemvArgs &a, int j, int R, uint32_t smem, uint32_
     x_lane[nb] = real ? smem + (uint32_t)(tok * xstride + (lane >> 3) * 16) : smem + a.L.zero_off;
     x_step[nb] = real ? 1u : 0u;
   }
-  if (*abort || !mbar_wait(bars + 8u * (2 * S), 0)) {  // x and metadata staged
-    *abort = 1;
-    bq_flag(BQ_FLAG_TIMEOUT);
+  // x and metadata staged; every wait is voted on, so the whole warp leaves
+  // together (mma.sync below needs every lane)
+  if (!__all_sync(0xffffffffu, (*abort == 0) && mbar_wait(bars + 8u * (2 * S), 0))) {
+    if (lane == 0) {
+      *abort = 1;
+      bq_flag(BQ_FLAG_TIMEOUT);
+    }
     return;
   }
   const uint32_t stile = smem + a.L.s_off + (j * 16 + r) * 4;
@@ -267,9 +271,11 @@ BQ_DEV void gemv_consume(const GemvArgs &a, int j, int R, uint32_t smem, uint32_
   int slot = 0, phase = 0;
   for (int i = 0; i < n; ++i) {
     const uint32_t full = bars + 8u * slot, empty = bars + 8u * (S + slot);
-    if (*abort || !mbar_wait(full, phase)) {
-      *abort = 1;
-      bq_flag(BQ_FLAG_TIMEOUT);
+    if (!__all_sync(0xffffffffu, (*abort == 0) && mbar_wait(full, phase))) {
+      if (lane == 0) {
+        *abort = 1;
+        bq_flag(BQ_FLAG_TIMEOUT);
+      }
       break;
     }
     const uint32_t wt = smem + (uint32_t)(a.L.ring_off + slot * 16384) + j * 512 + lane * 16;

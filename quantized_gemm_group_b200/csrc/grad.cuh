@@ -216,9 +216,12 @@ BQ_DEV void grad_consume(const GradArgs &a, int w, int64_t b0, int nblk, uint32_
   for (int i = 0; i < nblk; ++i) {
     const uint32_t st = smem + (uint32_t)((i % S) * a.L.sb);
     const uint32_t full = bars + 8u * (i % S), empty = bars + 8u * (S + i % S);
-    if (*abort || !mbar_wait(full, (i / S) & 1)) {
-      *abort = 1;
-      bq_flag(BQ_FLAG_TIMEOUT);
+    // the whole warp leaves together (mma.sync below needs every lane)
+    if (!__all_sync(0xffffffffu, (*abort == 0) && mbar_wait(full, (i / S) & 1))) {
+      if (lane == 0) {
+        *abort = 1;
+        bq_flag(BQ_FLAG_TIMEOUT);
+      }
       break;
     }
     const int rows = grad_block_rows(a.N, b0 + i);

@@ -333,9 +333,12 @@ quantize_tma_kernel(const __grid_constant__ CUtensorMap wmap, int64_t N, int64_t
   bool bad = false;
   for (int i = par; i < n; i += 2) {
     const int slot = i % stages;
-    if (*abort || !mbar_wait(bars + 8u * slot, (i / stages) & 1)) {
-      *abort = 1;
-      bq_flag(BQ_FLAG_TIMEOUT);
+    // the whole warp leaves together (the group reductions shuffle across lanes)
+    if (!__all_sync(0xffffffffu, (*abort == 0) && mbar_wait(bars + 8u * slot, (i / stages) & 1))) {
+      if (lane == 0) {
+        *abort = 1;
+        bq_flag(BQ_FLAG_TIMEOUT);
+      }
       break;
     }
     const int64_t su = blockIdx.x + (int64_t)i * gridDim.x;

@@ -53,3 +53,23 @@ __global__ void check_division_kernel(uint32_t s_begin, uint32_t s_end, unsigned
 }
 
 }  // namespace bq
+
+namespace bq {
+
+// One thread waits, through the bounded wait every kernel of the library
+// uses, on the first phase of an mbarrier that nothing ever arrives on.
+// After `limit` polls the wait gives up, the kernel records BQ_FLAG_TIMEOUT
+// and returns normally: the failure path of a bounded wait, exercised
+// without a hang or a fault.
+__global__ void bounded_wait_kernel(uint32_t limit) {
+  __shared__ __align__(8) unsigned long long bar;
+  const uint32_t b = smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    mbar_init(b, 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !mbar_wait(b, 0, limit)) bq_flag(BQ_FLAG_TIMEOUT);
+}
+
+}  // namespace bq

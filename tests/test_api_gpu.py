@@ -73,3 +73,60 @@ def test_degenerate_shapes():
     yn = bq.bq_linear(synth.activations(2, K, seed=14, device=DEV), pk, sc, ze, 0, 4, 128)
     assert yn.shape == (2, 0)
     assert bq.bq_device_status() == bq.BQ_OK
+
+
+def test_bounded_wait_gives_up_and_reports_timeout():
+    """The kernels' bounded wait, driven to expiry on a barrier phase nothing
+    completes: the kernel returns, the status reports BQ_ERR_TIMEOUT once,
+    and the context keeps working."""
+    assert bq.bq_device_status() == bq.BQ_OK
+    bq.bq_selftest_bounded_wait(256)
+    assert bq.bq_device_status() == bq.BQ_ERR_TIMEOUT
+    assert bq.bq_device_status() == bq.BQ_OK          # read and cleared
+    N, K = 256, 1024
+    W = synth.normal((N, K), 0.02, seed=11, dtype="f16", device=DEV)
+    pk, sc, ze = bq.bq_quantize(W, 4, 128, "interleaved")
+    x = synth.activations(2, K, seed=12, device=DEV)
+    y1 = bq.bq_linear(x, pk, sc, ze, N, 4, 128)
+    y2 = bq.bq_linear(x, pk, sc, ze, N, 4, 128)
+    torch.cuda.synchronize()
+    assert bq.bq_device_status() == bq.BQ_OK
+    assert torch.equal(y1, y2)
+    with pytest.raises(bq.BQError):
+        bq.bq_selftest_bounded_wait(0)
+
+
+def test_two_host_threads_two_streams():
+    """Two host threads call the library at once, each on its own stream:
+    results equal the sequential ones (kernel attributes are set per device
+    and kernel, options are atomic)."""
+    import threading
+    N, K = 2048, 4096
+    W = synth.normal((N, K), 0.02, seed=31, dtype="f16", device=DEV)
+    pk, sc, ze = bq.bq_quantize(W, 4, 128, "interleaved")
+    xs = [synth.activations(m, K, seed=40 + m, device=DEV) for m in (1, 16)]
+    ref = [bq.bq_linear(x, pk, sc, ze, N, 4, 128) for x in xs]
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream() for _ in xs]
+    got = [None, None]
+    errs = []
+
+    def run(t):
+        try:
+            with torch.cuda.stream(streams[t]):
+                ys = [bq.bq_linear(xs[t], pk, sc, ze, N, 4, 128, stream=streams[t]) for _ in range(20)]
+            streams[t].synchronize()
+            got[t] = ys
+        except Exception as e:  # noqa: BLE001
+            errs.append(e)
+
+    th = [threading.Thread(target=run, args=(t,)) for t in range(2)]
+    for t in th:
+        t.start()
+    for t in th:
+        t.join()
+    assert not errs, errs
+    assert bq.bq_device_status() == bq.BQ_OK
+    for t in range(2):
+        for y in got[t]:
+            assert torch.equal(y, ref[t])

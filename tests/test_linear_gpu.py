@@ -195,3 +195,54 @@ def test_fused_projections():
     x = synth.activations(4, K, seed=93, device=DEV)
     y = bq.bq_linear(x, pk2, sc2, ze2, N, 4, 128)
     check(y, oracle_y(x, Wc, 4, 128), torch.bfloat16)
+
+
+def oracle_y_mixed_rows(x: torch.Tensor, W: torch.Tensor, bit_map, rows: np.ndarray):
+    """fp64 oracle output of a mixed-width matrix for the given rows: each row
+    quantized with its 128-row block's width (rows quantize independently)."""
+    xf = O.decode_f64(synth.bits16(x), "bf16")
+    cols = []
+    for n in rows:
+        b = int(bit_map[int(n) // 128])
+        g = O.GROUP_OF_BITS[b]
+        c, s_, z = O.quantize(synth.bits16(W[int(n):int(n) + 1]), "f16", b, g)
+        cols.append(O.linear_f64(xf, c, s_, z, g)[:, 0])
+    return np.stack(cols, axis=1)
+
+
+@pytest.mark.parametrize("kind,N,K", [("channel", 14336, 4096), ("channel", 4096, 14336),
+                                      ("layer4", 14336, 4096), ("layer2", 4096, 14336)])
+def test_mixed_llama_sized_sampled(kind, N, K):
+    """Llama-3-8B-sized Channel-mix (25% of the 128-row blocks at 4 bits) and
+    Layer-mix (one width for the whole matrix) at M = 1 and 16, through the
+    mixed launch; the oracle checks sampled output channels of every width."""
+    W = synth.normal((N, K), 0.02, seed=N + 3, dtype="f16", device=DEV)
+    if kind == "channel":
+        bit_map = synth.channel_mix_map(N, seed=N + 5).tolist()
+    else:
+        bit_map = [4 if kind == "layer4" else 2] * (N // 128)
+    pk, sc, ze, bm = bq.bq_quantize_mixed(W, bit_map, "interleaved")
+    rng = np.random.default_rng(N)
+    rows = np.unique(np.concatenate([[0, 127, 128, N - 1], rng.choice(N, 44, replace=False)]))
+    x = synth.activations(16, K, seed=K + 9, device=DEV)
+    for M in (1, 16):
+        y = bq.bq_linear(x[:M].contiguous(), pk, sc, ze, N, bit_map_dev=bm)
+        y_ref = oracle_y_mixed_rows(x[:M].contiguous(), W, bit_map, rows)
+        check(y[:, torch.from_numpy(rows).to(DEV)], y_ref, torch.bfloat16)
+    assert bq.bq_device_status() == bq.BQ_OK
+
+
+def test_decode_split_blocks_many_shapes():
+    """The persistent decode kernel splits 128-row blocks between CTAs at
+    unit boundaries that depend on the shape; sweep shapes whose blocks are
+    split in different places (and a last partial block) against the oracle."""
+    for N, K in ((144, 4096), (1040, 2048), (3072, 1536), (256, 14336)):
+        W = synth.normal((N, K), 0.02, seed=N + K, dtype="f16", device=DEV)
+        for bits, group in ((4, 128), (2, 64)):
+            if K % (256 if bits == 4 else 512):
+                continue
+            pk, sc, ze = bq.bq_quantize(W, bits, group, "interleaved")
+            for M in (1, 16):
+                x = synth.activations(M, K, seed=M + N, device=DEV)
+                y = bq.bq_linear(x, pk, sc, ze, N, bits, group)
+                check(y, oracle_y(x, W, bits, group), torch.bfloat16)
