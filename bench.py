@@ -646,6 +646,59 @@ def gemm_numbers(Ms, bf16, bf16_sus, reps=10):
     return res
 
 
+def split_numbers(layers, bits, group, Ms, steps, world, rank, hbm):
+    """The decode stack split over the ranks by output channels (not measured
+    on more than one GPU here): each rank quantizes and keeps whole 128-row
+    blocks of every fused linear (shard.block_ranges), computes its rows of y,
+    and one NCCL all-gather per linear assembles y on every rank.  Eager
+    launches, timed with CUDA events over whole steps, max over ranks; value
+    is the whole stack's bytes (all ranks together) per step time.  With one
+    rank the gather is skipped."""
+    from quantized_gemm_group_b200 import shard
+    L = synth.LLAMA3_8B_LINEARS
+    fused = fused_shapes(layers)
+    lins = []
+    for (l, fname, N, K, mods) in fused:
+        parts = [synth.normal((L[m][1], K), 0.02, synth.weight_seed(l, m), "f16", "cuda") for m in mods]
+        W = torch.cat(parts) if len(parts) > 1 else parts[0]
+        lins.append(shard.ShardedLinear(W, bits, group, rank, world))
+        del W, parts
+    torch.cuda.synchronize()
+    if bq.bq_device_status() != bq.BQ_OK:
+        raise RuntimeError("quantizer reported a device error")
+    xs = {M: [synth.activations(M, K, seed=20000 * M + i, device="cuda") for i, (_, _, N, K, _) in enumerate(fused)]
+          for M in Ms}
+
+    def step(M):
+        for sl, x in zip(lins, xs[M]):
+            y = sl.local(x)
+            if world > 1:
+                shard.gather_rows(y, sl.ranges, rank)
+
+    res = {}
+    for M in Ms:
+        for _ in range(2):
+            step(M)
+        torch.cuda.synchronize()
+        barrier(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(steps):
+            step(M)
+        b.record()
+        b.synchronize()
+        t = max_over_ranks(a.elapsed_time(b) / 1e3 / steps, world)
+        byts = sum(linear_bytes(N, K, bits, group, M) for (_, _, N, K, _) in fused)
+        res[str(M)] = {"ms": round(t * 1e3, 4), "GBps": round(byts / t / 1e9, 1),
+                       "frac_of_measured_hbm_per_gpu": round(byts / t / 1e9 / hbm / world, 4)}
+    if bq.bq_device_status() != bq.BQ_OK:
+        raise RuntimeError("device error in the split stack")
+    del lins
+    torch.cuda.empty_cache()
+    return {"per_M": res, "ranks": world, "collective": "NCCL all_gather of y per linear" if world > 1 else "none",
+            "launches": "eager", "measured_on_hardware": "1 GPU only" if world == 1 else f"{world} GPUs"}
+
+
 def workload_config(args):
     """The workload both arms report (the reference arm times a bounded sample of it)."""
     bits = args.bits
@@ -741,6 +794,8 @@ def run_gpu(args, world, rank, local):
         torch.cuda.empty_cache()
     if not args.no_mixed:
         extra["mixed_stack"] = mixed_numbers(args.layers, (1, 16), hbm)
+    if args.split:
+        extra["split_stack"] = split_numbers(args.layers, bits, group, Ms, max(2, args.steps), world, rank, hbm)
     if not args.no_quant:
         extra["quantizer_8192x49152"] = quant_shape_numbers(hbm)
     if not args.no_gemm:
@@ -768,20 +823,30 @@ def run_gpu(args, world, rank, local):
 # CPU oracle (baseline and reference arm)
 # ---------------------------------------------------------------------------
 
-def oracle_sample(threads: int, layers_sample: int = 1, Ms=M_SET, bits=4):
-    """Time the CPU oracle's linear layer on a bounded sample of the stack:
-    the first `layers_sample` layers' linears (q/k/v and gate/up sharing
-    their input) at every M of the step."""
+def oracle_prepare(threads: int, layers_sample: int = 1, bits=4):
+    """Quantize (with the oracle) the first `layers_sample` layers' linears of
+    the stack on the host, q/k/v and gate/up each sharing their input."""
     from oracle import oracle as O  # test infrastructure, CPU baseline only
     group = 128 if bits == 4 else 64
-    total_bytes = 0
-    t_lin = 0.0
+    prep = []
     for (l, fname, N, K, mods) in fused_shapes(layers_sample):
         quant = []
         for m in mods:
             Nm = synth.LLAMA3_8B_LINEARS[m][1]
             W = synth.normal((Nm, K), 0.02, synth.weight_seed(l, m), "f16", "cpu")
             quant.append(O.quantize(synth.bits16(W), "f16", bits, group, threads=threads))
+        prep.append((N, K, mods, quant))
+    return prep, bits, group
+
+
+def oracle_sample(threads: int, prep, Ms=M_SET):
+    """Time the CPU oracle's linear layer over prepared linears at every M of
+    the step: (GB/s of weight traffic, seconds, bytes)."""
+    from oracle import oracle as O  # test infrastructure, CPU baseline only
+    lins, bits, group = prep
+    total_bytes = 0
+    t_lin = 0.0
+    for (N, K, mods, quant) in lins:
         for M in Ms:
             x = O.decode_f64(synth.bits16(synth.activations(M, K, seed=M + mods[0], device="cpu")), "bf16")
             t0 = time.perf_counter()
@@ -790,6 +855,30 @@ def oracle_sample(threads: int, layers_sample: int = 1, Ms=M_SET, bits=4):
             t_lin += time.perf_counter() - t0
             total_bytes += linear_bytes(N, K, bits, group, M)
     return total_bytes / t_lin / 1e9, t_lin, total_bytes
+
+
+def parity_sample(O, W, xt, y_ref, bits, group):
+    """The baseline's own oracle product (256 tokens `xt` x the first layer's
+    q weight `W`, both host tensors) against the library's on the GPU: the
+    decode kernel on the first token and the tensor-core kernel on all 256.
+    Per-token relative L2 error (the 2e-3 tolerance metric) and, for context,
+    the element-wise max of |y - y_ref| / max|y_ref|, both maxed over tokens.
+    Plain launches: the linear reads weights the quantizer has just written."""
+    yr = O.bf16_bits_to_f64(O.to_bf16_bits(y_ref))
+    mode = bq.bq_get_option(bq.BQ_OPT_LINEAR_OVERLAP)
+    bq.bq_set_option(bq.BQ_OPT_LINEAR_OVERLAP, 0)
+    pk, sc, ze = bq.bq_quantize(W.to("cuda"), bits, group, "interleaved")
+    x = xt.to("cuda")
+    out = {}
+    for name, xs, ref in (("decode_M1", x[:1], yr[:1]), ("prefill_M256", x, yr)):
+        y = bq.bq_linear(xs, pk, sc, ze, W.shape[0], bits, group).double().cpu().numpy()
+        l2 = float(np.max(np.linalg.norm(y - ref, axis=1) / np.linalg.norm(ref, axis=1)))
+        elem = float(np.max(np.max(np.abs(y - ref), axis=1) / np.max(np.abs(ref), axis=1)))
+        out[name] = {"rel_l2_max_over_tokens": float(f"{l2:.3e}"), "elementwise_max_rel": float(f"{elem:.3e}")}
+    assert bq.bq_device_status() == bq.BQ_OK
+    bq.bq_set_option(bq.BQ_OPT_LINEAR_OVERLAP, mode)
+    out["shape"] = f"{W.shape[0]}x{W.shape[1]} INT{bits} g{group}"
+    return out
 
 
 def cpu_baseline(args):
@@ -801,8 +890,11 @@ def cpu_baseline(args):
     from oracle import oracle as O  # test infrastructure, CPU baseline only
     threads = os.cpu_count() or 1
     bits, group = args.bits, (128 if args.bits == 4 else 64)
-    gbps, secs, byts = oracle_sample(threads, args.oracle_layers, bits=bits)
-    gbps1, secs1, byts1 = oracle_sample(1, 1, Ms=(1,), bits=bits)
+    prep = oracle_prepare(threads, args.oracle_layers, bits)
+    gbps, secs, byts = oracle_sample(threads, prep)
+    prep1 = (prep[0][:4], prep[1], prep[2])
+    gbps1, secs1, byts1 = oracle_sample(1, prep1, Ms=(1,))
+    del prep, prep1
     # quantizer: the first layer's seven weight matrices
     Ws = [synth.normal((N, K), 0.02, synth.weight_seed(0, m), "f16", "cpu")
           for m, (_, N, K) in enumerate(synth.LLAMA3_8B_LINEARS)]
@@ -818,12 +910,14 @@ def cpu_baseline(args):
     # prefill: 256 tokens against a 4096x4096 weight, per multiply-add
     W = Ws[0]
     c, sc, ze = O.quantize(synth.bits16(W), "f16", bits, group, threads=threads)
-    x = O.decode_f64(synth.bits16(synth.activations(256, W.shape[1], seed=3, device="cpu")), "bf16")
+    xt = synth.activations(256, W.shape[1], seed=3, device="cpu")
+    x = O.decode_f64(synth.bits16(xt), "bf16")
     t0 = time.perf_counter()
-    O.linear_f64(x, c, sc, ze, group, threads=threads)
+    y_ref = O.linear_f64(x, c, sc, ze, group, threads=threads)
     tg = time.perf_counter() - t0
     macs_per_s = 256 * W.shape[0] * W.shape[1] / tg
     big = 8192 * 49152 * 8192
+    parity = parity_sample(O, W, xt, y_ref, bits, group)
     return {"value": round(gbps, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
             "sample": f"first {args.oracle_layers} layer(s) x 4 linears (qkv, o, gate_up, down) x M in {{1,4,16}} "
                       f"({byts / 1e6:.1f} MB of weight traffic, {secs:.1f} s); fp64 linear over dequantized weights",
@@ -833,6 +927,7 @@ def cpu_baseline(args):
                           "cores": threads, "weights_per_s_single_core": round(Ws[0].numel() / tq1, 1),
                           "sample": f"first layer's 7 weight matrices ({nweights / 1e6:.0f} M weights, {tq:.1f} s; "
                                     f"one core: q 4096x4096, {tq1:.1f} s), INT{bits} g{group}"},
+            "parity_sample": parity,
             "prefill_extrapolated": {"TFLOPs": round(2 * macs_per_s / 1e12, 6), "cores": threads,
                                      "seconds_8192x49152_M8192": round(big / macs_per_s, 1),
                                      "sample": f"256 tokens x 4096x4096 fp64 ({tg:.1f} s), extrapolated per "
@@ -843,12 +938,13 @@ def run_reference(args, world, rank):
     if rank != 0:
         return None
     threads = os.cpu_count() or 1
-    for _ in range(args.warmup):
-        pass
-    times, gbps_all = [], []
+    times = []
     byts_step = None
+    prep = oracle_prepare(threads, args.reference_layers, args.bits)
+    for _ in range(args.warmup):
+        oracle_sample(threads, prep, Ms=(1,))
     for _ in range(max(1, args.steps)):
-        gbps, secs, byts = oracle_sample(threads, args.oracle_layers, bits=args.bits)
+        gbps, secs, byts = oracle_sample(threads, prep)
         times.append(secs)
         byts_step = byts
     t = statistics.median(times)
@@ -859,8 +955,8 @@ def run_reference(args, world, rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(args),
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
-                         "sample": f"first {args.oracle_layers} layer(s) x 4 linears (qkv, o, gate_up, down) "
-                                   f"x M in {{1,4,16}} per step"},
+                         "sample": f"first {args.reference_layers} layer(s) x 4 linears (qkv, o, gate_up, down) "
+                                   f"x M in {{1,4,16}} per step (quantized once, outside the timed steps)"},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -873,7 +969,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--bits", type=int, default=4, choices=[2, 4])
     ap.add_argument("--layers", type=int, default=synth.LLAMA3_8B_LAYERS)
-    ap.add_argument("--oracle-layers", type=int, default=4)
+    ap.add_argument("--oracle-layers", type=int, default=16,
+                    help="layers in the CPU baseline's timed oracle sample (about 10 s of CPU work)")
+    ap.add_argument("--reference-layers", type=int, default=1,
+                    help="layers per step of the reference arm (the oracle)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-quant", action="store_true")
     ap.add_argument("--quick", action="store_true", help="skip the per-shape breakdown")
@@ -882,6 +981,8 @@ def main():
     ap.add_argument("--no-mixed", action="store_true", help="skip the Layer-mix / Channel-mix decode stacks")
     ap.add_argument("--no-other-width", action="store_true",
                     help="skip the second stack at the other width (INT2 g64 when timing INT4)")
+    ap.add_argument("--split", action="store_true",
+                    help="also time the decode stack split over the ranks by output channels, y all-gathered")
     ap.add_argument("--overlap", type=int, default=2, choices=[0, 1, 2],
                     help="bq_linear launch overlap: 0 plain, 1 programmatic dependent launch, "
                          "2 PDL + weight streaming before the wait (weights are static here)")

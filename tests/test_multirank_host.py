@@ -20,7 +20,7 @@ CHILD = textwrap.dedent("""
     bench.barrier(world)
     t = bench.max_over_ranks(1.0 + rank, world)      # rank 1 is the slow one
     assert t == 2.0, t
-    args = type("A", (), {"steps": 1, "warmup": 0, "oracle_layers": 1, "bits": 4})()
+    args = type("A", (), {"steps": 1, "warmup": 0, "oracle_layers": 1, "reference_layers": 1, "bits": 4})()
     out = bench.run_reference(args, world, rank) if rank == 1 else None
     assert out is None                               # only rank 0 runs the reference arm
     import torch.distributed as dist
