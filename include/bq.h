@@ -290,6 +290,22 @@ bq_status bq_check_division(uint32_t s_bits_begin, uint32_t s_bits_end, int refi
                             unsigned long long *result, void *stream);
 
 /*
+ * bq_check_const_division: diagnostic.  The quantizer computes the group
+ * scale s = (hi - lo) / (2^b - 1) (and the symmetric scale max|x| /
+ * (2^(b-1) - 1)) by the same refinement with the constant r = RN(1/D), for
+ * 2^-100 <= |x| <= 2^120, and by the IEEE division outside that range.  This
+ * entry point compares that quotient bit for bit against the IEEE division
+ * by `divisor` (3, 7 or 15; others return BQ_ERR_UNSUPPORTED) for every fp32
+ * bit pattern in [x_bits_begin, x_bits_end) (NaN inputs compare equal when
+ * both results are NaN).
+ *   result  DEVICE array of 4 uint64, zeroed by the caller: [0] mismatches,
+ *           [1] values checked, [2] bit pattern of the first mismatch found,
+ *           [3] the divisor it was found for.
+ */
+bq_status bq_check_const_division(int divisor, uint32_t x_bits_begin, uint32_t x_bits_end,
+                                  unsigned long long *result, void *stream);
+
+/*
  * bq_selftest_bounded_wait: diagnostic of the failure path of the kernels'
  * bounded waits.  Launches one small kernel on `stream` that waits, with the
  * same routine every kernel of the library uses, on a shared-memory barrier

@@ -34,6 +34,7 @@ EXPORTS = (
     "bq_packed_bytes", "bq_group_count", "bq_mixed_offsets", "bq_quantize", "bq_quantize_symmetric",
     "bq_quantize_mixed",
     "bq_dequantize", "bq_fake_quantize", "bq_linear", "bq_linear_grad_input", "bq_check_division",
+    "bq_check_const_division",
     "bq_selftest_bounded_wait", "bq_set_option", "bq_get_option", "bq_device_status",
     "bq_status_string", "bq_version",
 )
@@ -82,6 +83,8 @@ def lib(path: str | None = None):
     L.bq_linear_grad_input.restype = i32
     L.bq_check_division.argtypes = [ctypes.c_uint32, ctypes.c_uint32, i32, vp, vp]
     L.bq_check_division.restype = i32
+    L.bq_check_const_division.argtypes = [i32, ctypes.c_uint32, ctypes.c_uint32, vp, vp]
+    L.bq_check_const_division.restype = i32
     L.bq_selftest_bounded_wait.argtypes = [ctypes.c_uint32, vp]
     L.bq_selftest_bounded_wait.restype = i32
     L.bq_set_option.argtypes = [i32, i32]
@@ -236,6 +239,15 @@ def bq_check_division(s_bits_begin: int, s_bits_end: int, refinements: int = 2, 
     res = torch.zeros(4, dtype=torch.int64, device="cuda")
     _check("bq_check_division", lib().bq_check_division(s_bits_begin, s_bits_end, refinements, _ptr(res),
                                                         _stream(stream)))
+    torch.cuda.synchronize()
+    return tuple(int(v) for v in res.cpu())
+
+
+def bq_check_const_division(divisor: int, x_bits_begin: int, x_bits_end: int, stream=None):
+    """Returns (mismatches, values checked, first bad x bits, its divisor)."""
+    res = torch.zeros(4, dtype=torch.int64, device="cuda")
+    _check("bq_check_const_division", lib().bq_check_const_division(divisor, x_bits_begin, x_bits_end, _ptr(res),
+                                                                    _stream(stream)))
     torch.cuda.synchronize()
     return tuple(int(v) for v in res.cpu())
 

@@ -140,7 +140,7 @@ bq_status quantize_tma(const uint16_t *W, int64_t N, int64_t K, uint8_t *packed,
                        cudaStream_t st) {
   constexpr int U = UnitGeom<BITS, G>::U;
   constexpr int SU = (U / 64) * 8192;
-  constexpr int kBudget = 113 * 1024;
+  constexpr int kBudget = (227 * 1024) / qt_ctas_per_sm<G>() - 1024;  // shared memory per CTA
   auto kern = quantize_tma_kernel<WT, BITS, G, SCHEME>;
   if (!ensure_smem<quantize_tma_kernel<WT, BITS, G, SCHEME>>(kBudget)) return BQ_ERR_CUDA;
   int stages = (kBudget - 1024 - 16) / (SU + 16);
@@ -150,7 +150,7 @@ bq_status quantize_tma(const uint16_t *W, int64_t N, int64_t K, uint8_t *packed,
   CUtensorMap map;
   if (!make_map_2d(&map, W, N, K, WT == 1, 64, 64)) return BQ_ERR_CUDA;
   const int64_t nsu = ((N + 63) / 64) * (K / U);
-  int64_t grid = 2 * (int64_t)sm_count();
+  int64_t grid = qt_ctas_per_sm<G>() * (int64_t)sm_count();
   if (grid > nsu) grid = nsu;
   kern<<<(unsigned)grid, kQtThreads, smem, st>>>(map, N, K, stages, packed, scales, zeros);
   return launch_status();
@@ -802,6 +802,19 @@ bq_status bq_check_division(uint32_t s_bits_begin, uint32_t s_bits_end, int refi
   const int64_t grid = sm_count() * 8;
   if (refinements == 1) check_division_kernel<1><<<grid, kThreads, 0, st>>>(s_bits_begin, s_bits_end, result);
   else if (refinements == 2) check_division_kernel<2><<<grid, kThreads, 0, st>>>(s_bits_begin, s_bits_end, result);
+  else return BQ_ERR_UNSUPPORTED;
+  return launch_status();
+}
+
+bq_status bq_check_const_division(int divisor, uint32_t x_bits_begin, uint32_t x_bits_end,
+                                  unsigned long long *result, void *stream) {
+  if (!result) return BQ_ERR_NULL;
+  if (x_bits_end <= x_bits_begin) return BQ_ERR_SHAPE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t grid = sm_count() * 8;
+  if (divisor == 15) check_const_division_kernel<15><<<grid, kThreads, 0, st>>>(x_bits_begin, x_bits_end, result);
+  else if (divisor == 7) check_const_division_kernel<7><<<grid, kThreads, 0, st>>>(x_bits_begin, x_bits_end, result);
+  else if (divisor == 3) check_const_division_kernel<3><<<grid, kThreads, 0, st>>>(x_bits_begin, x_bits_end, result);
   else return BQ_ERR_UNSUPPORTED;
   return launch_status();
 }

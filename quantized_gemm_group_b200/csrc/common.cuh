@@ -129,8 +129,30 @@ BQ_DEV int round_even_small(float t) {
   return __float_as_int(__fadd_rn(t, kRoundMagic)) - kRoundMagicBits;
 }
 
+// RN(x / D) for the small constant divisors 2^b - 1 and 2^(b-1) - 1: the
+// refined quotient above with r = RN(1/D) (a constant), where its residuals
+// stay normal (2^-100 <= |x| <= 2^120); the IEEE division elsewhere.
+template <int D>
+BQ_DEV float div_const(float x) {
+  static_assert(D == 1 || D == 3 || D == 7 || D == 15, "no reciprocal constant for this divisor");
+  if (D == 1) return x;
+  // RN(1/15), RN(1/3), RN(1/7) in fp32 (0x3d888889, 0x3eaaaaab, 0x3e124925)
+  constexpr float kInv = (D == 15) ? 0x1.111112p-4f : (D == 3) ? 0x1.555556p-2f : 0x1.24924ap-3f;
+  const float ax = fabsf(x);
+  if (ax >= 0x1p-100f && ax <= 0x1p120f) return div_refined(x, (float)D, kInv);
+  return __fdiv_rn(x, (float)D);
+}
+
+// RN(x / s) given r = RN(1/s): the refined quotient when s lies in
+// [2^-60, 2^60] (`fast`), where every quotient whose rounding to an integer
+// matters keeps its residuals normal; the IEEE division otherwise.
+BQ_DEV float div_group(float x, float s, float r, bool fast) {
+  return fast ? div_refined(x, s, r) : __fdiv_rn(x, s);
+}
+
 // Per-group quantization parameters, computed exactly as the reading of the
-// method prescribes (range widened to contain 0, fp32 IEEE steps).
+// method prescribes (range widened to contain 0, correctly rounded fp32
+// steps: every quotient below equals the IEEE division's).
 struct GroupParams {
   float s;       // stored scale (0 for an all-zero group)
   float sd;      // divisor used for the codes (1 for an all-zero group: 0/1 = 0)
@@ -152,7 +174,7 @@ BQ_DEV GroupParams group_params_sym(float mn, float mx) {
   GroupParams p;
   p.bad = !(fabsf(mn) <= 3.402823466e38f) || !(fabsf(mx) <= 3.402823466e38f);
   const float amax = fmaxf(fabsf(mn), fabsf(mx));
-  const float s = __fdiv_rn(amax, (float)(ZC - 1));
+  const float s = div_const<ZC - 1>(amax);
   p.bad |= !(s <= 3.402823466e38f);
   p.z = ZC;
   p.zc = ZC - kRoundMagicBits;
@@ -168,7 +190,7 @@ BQ_DEV GroupParams group_params_sym(float mn, float mx) {
   p.sd = s;
   p.fast = (s >= 8.67361738e-19f) && (s <= 1.15292150e18f);  // 2^-60 .. 2^60
   p.r = __frcp_rn(s);
-  p.clamp = __float2int_rn(__fdiv_rn(amax, s)) + ZC > QMAX;
+  p.clamp = __float2int_rn(div_group(amax, s, p.r, p.fast)) + ZC > QMAX;
   return p;
 }
 
@@ -180,7 +202,7 @@ BQ_DEV GroupParams group_params(float mn, float mx) {
   p.bad = !(fabsf(mn) <= 3.402823466e38f) || !(fabsf(mx) <= 3.402823466e38f);
   float lo = fminf(mn, 0.0f);
   float hi = fmaxf(mx, 0.0f);
-  float s = __fdiv_rn(__fsub_rn(hi, lo), (float)QMAX);
+  float s = div_const<QMAX>(__fsub_rn(hi, lo));
   p.bad |= !(s <= 3.402823466e38f);
   if (p.bad || s == 0.0f) {
     // all-zero group: s = 0, z = 0 and every x is +-0, so x / 1 rounds to 0
@@ -196,24 +218,21 @@ BQ_DEV GroupParams group_params(float mn, float mx) {
   }
   p.s = s;
   p.sd = s;
-  p.z = __float2int_rn(__fdiv_rn(-lo, s));
-  p.zc = p.z - kRoundMagicBits;
   p.fast = (s >= 8.67361738e-19f) && (s <= 1.15292150e18f);  // 2^-60 .. 2^60
   p.r = __frcp_rn(s);
+  p.z = __float2int_rn(div_group(-lo, s, p.r, p.fast));
+  p.zc = p.z - kRoundMagicBits;
   // Codes are monotone in x, so only the largest element can overflow:
   // round(hi / s) + z > 2^b - 1 decides whether this group needs the clamp.
-  p.clamp = __float2int_rn(__fdiv_rn(hi, s)) + p.z > QMAX;
+  p.clamp = __float2int_rn(div_group(hi, s, p.r, p.fast)) + p.z > QMAX;
   return p;
 }
 
-// Codes of two elements of one group.
-// code = min(round(x/s) + z, 2^b - 1); round(x/s) + z >= 0 always holds
-// (x >= lo gives round(x/s) >= round(lo/s) = -z), and round(x/s) + z can
-// exceed 2^b - 1 only in groups flagged `clamp`.  The unsigned min also keeps
-// a bad group's garbage inside its own field.  ALWAYS_FAST: fp16 inputs,
-// whose scales always lie in [2^-28, 2^16].
-template <int QMAX, bool ALWAYS_FAST, bool CLAMP>
-BQ_DEV uint2 code_pair(float2 v, const GroupParams &p) {
+// x / s rounded to an integer (ties to even) for two elements, still carrying
+// the 1.5 * 2^23 magic: the low bits of each result's bit pattern minus
+// kRoundMagicBits are round(x / s).  ALWAYS_FAST as in code_pair.
+template <bool ALWAYS_FAST>
+BQ_DEV float2 rounded_quotients(float2 v, const GroupParams &p) {
   float2 t;
   if (ALWAYS_FAST || p.fast) {
     const float2 r2 = make_float2(p.r, p.r), ns2 = make_float2(-p.sd, -p.sd);
@@ -225,7 +244,18 @@ BQ_DEV uint2 code_pair(float2 v, const GroupParams &p) {
   } else {
     t = make_float2(__fdiv_rn(v.x, p.sd), __fdiv_rn(v.y, p.sd));
   }
-  const float2 m = __fadd2_rn(t, make_float2(kRoundMagic, kRoundMagic));
+  return __fadd2_rn(t, make_float2(kRoundMagic, kRoundMagic));
+}
+
+// Codes of two elements of one group.
+// code = min(round(x/s) + z, 2^b - 1); round(x/s) + z >= 0 always holds
+// (x >= lo gives round(x/s) >= round(lo/s) = -z), and round(x/s) + z can
+// exceed 2^b - 1 only in groups flagged `clamp`.  The unsigned min also keeps
+// a bad group's garbage inside its own field.  ALWAYS_FAST: fp16 inputs,
+// whose scales always lie in [2^-28, 2^16].
+template <int QMAX, bool ALWAYS_FAST, bool CLAMP>
+BQ_DEV uint2 code_pair(float2 v, const GroupParams &p) {
+  const float2 m = rounded_quotients<ALWAYS_FAST>(v, p);
   uint32_t a = (uint32_t)(__float_as_int(m.x) + p.zc);
   uint32_t b = (uint32_t)(__float_as_int(m.y) + p.zc);
   if (CLAMP) {

@@ -155,7 +155,13 @@ BQ_DEV void load_unit(UnitRegs<BITS, G> &u, const uint16_t *__restrict__ W, int6
   }
 }
 
-// Codes of one (row half, group) of the unit ORed into the lane's tile words.
+// Codes of one (row half, group) of the unit added into the lane's tile
+// words (every code owns its own bit field, so adding is ORing).  A group
+// that needs no clamp adds each rounded quotient's raw bit pattern times
+// 2^(bit position) -- one integer multiply-add per code, off the ALU pipe --
+// and then, once per word, (z - kRoundMagicBits) times the sum of its
+// positions' 2^(bit position): modulo 2^32 the magic cancels and every field
+// receives round(x / s) + z.  A clamp group packs clamped codes directly.
 template <int WT, int BITS, int G, bool CLAMP>
 BQ_DEV void codes_of_group(const UnitRegs<BITS, G> &u, int h, int gi, const GroupParams &p,
                            uint32_t (&word)[UnitGeom<BITS, G>::TILES][4]) {
@@ -166,16 +172,37 @@ BQ_DEV void codes_of_group(const UnitRegs<BITS, G> &u, int h, int gi, const Grou
   for (int jj = 0; jj < UG::RUNS_PER_G; ++jj) {
     const int j = gi * UG::RUNS_PER_G + jj;
     const int t = j / UG::RUNS_PER_TILE, jt = j % UG::RUNS_PER_TILE;
+    uint32_t &w = word[t][tile_word<BITS>(jt)];
+    if (CLAMP) {
 #pragma unroll
-    for (int hp = 0; hp < 2; ++hp) {
-      const uint2 q = code_pair<QMAX, WT == 0, CLAMP>(E::pair(u.x[h][j][hp]), p);
-      word[t][tile_word<BITS>(jt)] |= __byte_perm(q.x, q.y, 0x5410) << tile_bit<BITS>(jt, h, hp);
+      for (int hp = 0; hp < 2; ++hp) {
+        const uint2 q = code_pair<QMAX, WT == 0, true>(E::pair(u.x[h][j][hp]), p);
+        w += __byte_perm(q.x, q.y, 0x5410) << tile_bit<BITS>(jt, h, hp);
+      }
+    } else {
+      uint32_t posmask = 0;
+#pragma unroll
+      for (int hp = 0; hp < 2; ++hp) {
+        const int bp = tile_bit<BITS>(jt, h, hp);
+        const float2 m = rounded_quotients<WT == 0>(E::pair(u.x[h][j][hp]), p);
+        w += __float_as_uint(m.x) * (1u << bp);
+        w += __float_as_uint(m.y) * (1u << (bp + 16));
+        posmask += (1u << bp) + (1u << (bp + 16));
+      }
+      w += (uint32_t)p.zc * posmask;
     }
   }
 }
 
 // Quantize one loaded unit: rows row0..row0+15, columns col0..col0+U-1 of an
 // N x K matrix; `packed`, `scales`, `zeros` are that matrix's own.
+// The four lanes of a quad share one row (r = lane / 4) and hold C = 2 x NG
+// (row half, group) combinations of it.  Their min / max are reduced across
+// the quad by a reduce-scatter (exchange with lane ^ 2, then lane ^ 1, each
+// step keeping half of the list while it is longer than one), so each lane
+// ends up with max(1, C / 4) whole combinations, computes their parameters,
+// stores their scale and zero, and the codes of every combination take the
+// parameters from the lane that computed them by shuffle.
 template <int WT, int BITS, int G, int SCHEME = 0>
 BQ_DEV bool quantize_unit(const UnitRegs<BITS, G> &u, int64_t N, int64_t K, int64_t row0, int64_t col0,
                           uint8_t *__restrict__ packed, float *__restrict__ scales,
@@ -183,14 +210,18 @@ BQ_DEV bool quantize_unit(const UnitRegs<BITS, G> &u, int64_t N, int64_t K, int6
   using UG = UnitGeom<BITS, G>;
   using E = Elem<WT>;
   constexpr int QMAX = (1 << BITS) - 1;
+  constexpr int NG = UG::NG;
+  constexpr int C = 2 * NG;                  // combinations (h, gi), k = h * NG + gi
+  constexpr int HALF = C / 2;
+  constexpr int LF = (C >= 4) ? C / 4 : 1;   // combinations finished per lane
   const int r = lane >> 2, c = lane & 3;
 
-  bool bad_any = false;
-  GroupParams gp[2][UG::NG];
+  // this lane's partial min / max of every combination
+  float vmn[C], vmx[C];
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
 #pragma unroll
-    for (int gi = 0; gi < UG::NG; ++gi) {
+    for (int gi = 0; gi < NG; ++gi) {
       uint32_t mn2 = u.x[h][gi * UG::RUNS_PER_G][0], mx2 = mn2;
 #pragma unroll
       for (int j = gi * UG::RUNS_PER_G; j < (gi + 1) * UG::RUNS_PER_G; ++j) {
@@ -200,14 +231,49 @@ BQ_DEV bool quantize_unit(const UnitRegs<BITS, G> &u, int64_t N, int64_t K, int6
           mx2 = E::max2(mx2, u.x[h][j][hp]);
         }
       }
-      float mn = fmin_nan(E::lo(mn2), E::hi(mn2));
-      float mx = fmax_nan(E::lo(mx2), E::hi(mx2));
-      mn = fmin_nan(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
-      mx = fmax_nan(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-      mn = fmin_nan(mn, __shfl_xor_sync(0xffffffffu, mn, 2));
-      mx = fmax_nan(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      gp[h][gi] = group_params<QMAX, SCHEME>(mn, mx);
-      bad_any |= gp[h][gi].bad;
+      vmn[h * NG + gi] = fmin_nan(E::lo(mn2), E::hi(mn2));
+      vmx[h * NG + gi] = fmax_nan(E::lo(mx2), E::hi(mx2));
+    }
+  }
+  // step 1: with lane ^ 2, keep the upper half of the list if lane bit 1 is set
+  const bool up2 = (c & 2) != 0;
+  float amn[HALF], amx[HALF];
+#pragma unroll
+  for (int i = 0; i < HALF; ++i) {
+    const float kmn = up2 ? vmn[HALF + i] : vmn[i], smn = up2 ? vmn[i] : vmn[HALF + i];
+    const float kmx = up2 ? vmx[HALF + i] : vmx[i], smx = up2 ? vmx[i] : vmx[HALF + i];
+    amn[i] = fmin_nan(kmn, __shfl_xor_sync(0xffffffffu, smn, 2));
+    amx[i] = fmax_nan(kmx, __shfl_xor_sync(0xffffffffu, smx, 2));
+  }
+  // step 2: with lane ^ 1, halve again (or, with one left, reduce it)
+  float fmn[LF], fmx[LF];
+  const bool up1 = (c & 1) != 0;
+#pragma unroll
+  for (int i = 0; i < LF; ++i) {
+    if (HALF >= 2) {
+      const float kmn = up1 ? amn[LF + i] : amn[i], smn = up1 ? amn[i] : amn[LF + i];
+      const float kmx = up1 ? amx[LF + i] : amx[i], smx = up1 ? amx[i] : amx[LF + i];
+      fmn[i] = fmin_nan(kmn, __shfl_xor_sync(0xffffffffu, smn, 1));
+      fmx[i] = fmax_nan(kmx, __shfl_xor_sync(0xffffffffu, smx, 1));
+    } else {
+      fmn[i] = fmin_nan(amn[0], __shfl_xor_sync(0xffffffffu, amn[0], 1));
+      fmx[i] = fmax_nan(amx[0], __shfl_xor_sync(0xffffffffu, amx[0], 1));
+    }
+  }
+  // combinations held: base + i, base from the two lane bits
+  const int base = (up2 ? HALF : 0) + ((HALF >= 2 && up1) ? LF : 0);
+  bool bad_any = false;
+  GroupParams own[LF];
+  const int64_t GK = K / G;
+#pragma unroll
+  for (int i = 0; i < LF; ++i) {
+    own[i] = group_params<QMAX, SCHEME>(fmn[i], fmx[i]);
+    bad_any |= own[i].bad;
+    if (HALF >= 2 || !up1) {  // with C = 2, lanes c and c ^ 1 hold the same combination
+      const int k = base + i, h = k / NG, gi = k % NG;
+      const int64_t idx = il_meta_index(row0 + r + 8 * h, col0 / G + gi, N, GK);
+      scales[idx] = own[i].s;
+      zeros[idx] = (uint8_t)own[i].z;
     }
   }
 
@@ -217,29 +283,27 @@ BQ_DEV bool quantize_unit(const UnitRegs<BITS, G> &u, int64_t N, int64_t K, int6
 #pragma unroll
     for (int i = 0; i < 4; ++i) word[t][i] = 0u;
 #pragma unroll
-  for (int h = 0; h < 2; ++h)
-#pragma unroll
-    for (int gi = 0; gi < UG::NG; ++gi) {
-      if (gp[h][gi].clamp) codes_of_group<WT, BITS, G, true>(u, h, gi, gp[h][gi], word);
-      else codes_of_group<WT, BITS, G, false>(u, h, gi, gp[h][gi], word);
-    }
+  for (int k = 0; k < C; ++k) {
+    // the lane of this quad that finished combination k, and its slot there
+    const int src_c = (k >= HALF ? 2 : 0) + ((HALF >= 2 && (k % HALF) >= LF) ? 1 : 0);
+    const int slot = (HALF >= 2) ? (k % HALF) % LF : 0;
+    const int src = (lane & ~3) | src_c;
+    const GroupParams &o = own[slot];
+    GroupParams p;
+    p.r = __shfl_sync(0xffffffffu, o.r, src);
+    p.sd = __shfl_sync(0xffffffffu, o.sd, src);
+    p.zc = __shfl_sync(0xffffffffu, o.zc, src);
+    const int fl = __shfl_sync(0xffffffffu, (o.fast ? 1 : 0) | (o.clamp ? 2 : 0), src);
+    p.fast = (fl & 1) != 0;
+    p.clamp = (fl & 2) != 0;
+    const int h = k / NG, gi = k % NG;
+    if (p.clamp) codes_of_group<WT, BITS, G, true>(u, h, gi, p, word);
+    else codes_of_group<WT, BITS, G, false>(u, h, gi, p, word);
+  }
 #pragma unroll
   for (int t = 0; t < UG::TILES; ++t) {
     const int64_t off = il_tile_offset(row0 / 16, col0 / UG::T + t, N, K, BITS);
     st_v4(packed + off + lane * 16, make_uint4(word[t][0], word[t][1], word[t][2], word[t][3]));
-  }
-
-  if (c == 0) {
-    const int64_t GK = K / G;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-#pragma unroll
-      for (int gi = 0; gi < UG::NG; ++gi) {
-        const int64_t idx = il_meta_index(row0 + r + 8 * h, col0 / G + gi, N, GK);
-        scales[idx] = gp[h][gi].s;
-        zeros[idx] = (uint8_t)gp[h][gi].z;
-      }
-    }
   }
   return bad_any;
 }
@@ -257,6 +321,9 @@ BQ_DEV bool quantize_unit(const UnitRegs<BITS, G> &u, int64_t N, int64_t K, int6
 // ones, warp w quantizing row tile w % 4.  CTAs stride over the super-units.
 constexpr int kQtConsumers = 8;
 constexpr int kQtThreads = 32 * (kQtConsumers + 1);
+// CTAs per SM: three where the unit fits 72 registers without spilling
+// (groups 32 to 128; measured on B200: 2-10% faster than two), else two.
+template <int G> constexpr int qt_ctas_per_sm() { return (G >= 32 && G <= 128) ? 3 : 2; }
 
 template <int BITS, int G>
 BQ_DEV void load_unit_smem(UnitRegs<BITS, G> &u, uint32_t su, int t, int lane) {
@@ -278,7 +345,7 @@ BQ_DEV void load_unit_smem(UnitRegs<BITS, G> &u, uint32_t su, int t, int lane) {
 }
 
 template <int WT, int BITS, int G, int SCHEME = 0>
-__global__ void __launch_bounds__(kQtThreads, 2)
+__global__ void __launch_bounds__(kQtThreads, qt_ctas_per_sm<G>())
 quantize_tma_kernel(const __grid_constant__ CUtensorMap wmap, int64_t N, int64_t K, int stages,
                     uint8_t *__restrict__ packed, float *__restrict__ scales, uint8_t *__restrict__ zeros) {
   using UG = UnitGeom<BITS, G>;

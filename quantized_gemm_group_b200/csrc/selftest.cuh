@@ -52,6 +52,27 @@ __global__ void check_division_kernel(uint32_t s_begin, uint32_t s_end, unsigned
   atomicAdd(result + 1, checked);
 }
 
+// The quantizer's division by the constant number of levels (div_const):
+// every fp32 bit pattern in [x_begin, x_end) against the IEEE division by D.
+template <int D>
+__global__ void check_const_division_kernel(uint32_t x_begin, uint32_t x_end, unsigned long long *result) {
+  unsigned long long bad = 0, checked = 0;
+  for (uint64_t xb = x_begin + (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; xb < x_end;
+       xb += (uint64_t)gridDim.x * blockDim.x) {
+    const float x = __uint_as_float((uint32_t)xb);
+    const float ref = __fdiv_rn(x, (float)D);
+    const float got = div_const<D>(x);
+    // identical bits (NaN inputs: any NaN)
+    if (__float_as_uint(ref) != __float_as_uint(got) && !(ref != ref && got != got)) {
+      if (bad == 0 && atomicCAS(result + 2, 0ull, (unsigned long long)xb) == 0ull) result[3] = D;
+      ++bad;
+    }
+    ++checked;
+  }
+  atomicAdd(result + 0, bad);
+  atomicAdd(result + 1, checked);
+}
+
 }  // namespace bq
 
 namespace bq {
