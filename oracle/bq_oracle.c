@@ -32,6 +32,12 @@
  *   R4  scales are fp32, zeros are uint8.
  *   R5  groups run along the input dimension K inside one output row.
  *   R8  a non-finite input, or a group whose fp32 scale overflows, is an error.
+ *   R14 fp16 group scales (a storage format of the same scheme): s is
+ *       computed as in R1-R3, then rounded to the nearest binary16 (ties to
+ *       even); a positive s that rounds to zero takes the smallest positive
+ *       binary16 (2^-24), one that rounds to infinity is an error (R8).  z and
+ *       the codes are then computed from the stored binary16 scale exactly as
+ *       R3 prescribes, so (q - z) * s16 is the reconstruction.
  *
  * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -fPIC -shared.
  * -ffp-contract=off keeps every multiply and add separately rounded, so the
@@ -81,6 +87,38 @@ float bqo_bf16_to_f32(uint16_t h)
     return v;
 }
 
+/* binary32 -> binary16, round to nearest, ties to even, from the format's
+ * definition: 10 fraction bits, exponent bias 15, subnormals below 2^-14
+ * with a fixed step of 2^-24, values at or above 65520 (halfway between the
+ * largest finite 65504 and 2^16) round to infinity. */
+uint16_t bqo_f32_to_f16(float v)
+{
+    uint16_t sign = signbit(v) ? 0x8000u : 0u;
+    float a = fabsf(v);
+    if (isnan(v)) return (uint16_t)(sign | 0x7e00u);
+    if (a >= 65520.0f) return (uint16_t)(sign | 0x7c00u);
+    /* the step (unit in the last place) of binary16 at a */
+    int e;
+    frexpf(a, &e);                     /* a = m * 2^e, 0.5 <= m < 1 */
+    int ulp_exp = e - 11;              /* 11 significant bits */
+    if (ulp_exp < -24) ulp_exp = -24;  /* subnormal step */
+    /* a / step is exact in binary32 (a scaled by a power of two); round it
+     * to an integer, half to even */
+    float n = nearbyintf(ldexpf(a, -ulp_exp));
+    double r = ldexp((double)n, ulp_exp);   /* the rounded magnitude, exact */
+    if (r == 0.0) return sign;
+    int re;
+    frexp(r, &re);
+    if (re - 1 < -14) {                /* subnormal: fraction = r / 2^-24 */
+        return (uint16_t)(sign | (uint16_t)ldexp(r, 24));
+    }
+    if (re - 1 > 15) return (uint16_t)(sign | 0x7c00u);
+    /* normal: r = (1 + f/1024) * 2^(re-1) */
+    uint16_t exp_field = (uint16_t)(re - 1 + 15);
+    uint16_t frac = (uint16_t)(ldexp(r, -(re - 1) + 10) - 1024.0);
+    return (uint16_t)(sign | (exp_field << 10) | frac);
+}
+
 static float decode(uint16_t h, int wtype)
 {
     return wtype == 0 ? bqo_f16_to_f32(h) : bqo_bf16_to_f32(h);
@@ -90,8 +128,10 @@ static float decode(uint16_t h, int wtype)
 /* One group: [GB] MinMax quantizer with [4BG] s.2.2 arithmetic.        */
 /* ------------------------------------------------------------------ */
 
-int bqo_quantize_group(const float *x, int g, int bits,
-                       float *s_out, int *z_out, uint8_t *q_out)
+/* f16_scale = 1: reading R14, the scale stored as binary16 (one rounding
+ * step inserted after s is computed; z and the codes then use it). */
+static int quantize_group_minmax(const float *x, int g, int bits, int f16_scale,
+                                 float *s_out, int *z_out, uint8_t *q_out)
 {
     if (g <= 0 || bits < 1 || bits > 8) return BQO_ERR_ARG;
     const int qmax = (1 << bits) - 1;
@@ -120,6 +160,13 @@ int bqo_quantize_group(const float *x, int g, int bits,
         return BQO_OK;
     }
 
+    /* R14: round the scale to binary16 and work with the stored value */
+    if (f16_scale) {
+        s = bqo_f16_to_f32(bqo_f32_to_f16(s));
+        if (s == 0.0f) s = ldexpf(1.0f, -24);
+        if (!isfinite(s)) return BQO_ERR_NONFINITE;
+    }
+
     /* z = round(-min / s), half to even (the default rounding mode) */
     float zq = -lo / s;
     int z = (int)nearbyintf(zq);
@@ -136,6 +183,19 @@ int bqo_quantize_group(const float *x, int g, int bits,
     *s_out = s;
     *z_out = z;
     return BQO_OK;
+}
+
+int bqo_quantize_group(const float *x, int g, int bits,
+                       float *s_out, int *z_out, uint8_t *q_out)
+{
+    return quantize_group_minmax(x, g, bits, 0, s_out, z_out, q_out);
+}
+
+/* R14: the MinMax scheme with the scale stored as binary16. */
+int bqo_quantize_group_s16(const float *x, int g, int bits,
+                           float *s_out, int *z_out, uint8_t *q_out)
+{
+    return quantize_group_minmax(x, g, bits, 1, s_out, z_out, q_out);
 }
 
 /* Symmetric abs-max scheme ("大模型量化实战", section 2.3: s = x_absmax /
@@ -193,12 +253,14 @@ int bqo_quantize(const uint16_t *W, int wtype, int64_t rows, int64_t cols,
 }
 
 /* scheme 0: asymmetric MinMax (bqo_quantize_group); 1: symmetric abs-max
- * (bqo_quantize_group_sym). */
+ * (bqo_quantize_group_sym); 2: asymmetric MinMax with binary16 scales
+ * (bqo_quantize_group_s16; the scales are written as the binary32 values of
+ * the stored binary16 numbers). */
 int bqo_quantize_scheme(const uint16_t *W, int wtype, int64_t rows, int64_t cols,
                         int bits, int group, int scheme, int64_t r0, int64_t r1,
                         uint8_t *codes, float *scales, uint8_t *zeros)
 {
-    if (scheme != 0 && scheme != 1) return BQO_ERR_ARG;
+    if (scheme < 0 || scheme > 2) return BQO_ERR_ARG;
     if (group <= 0 || cols % group != 0 || r0 < 0 || r1 > rows) return BQO_ERR_ARG;
     if (group > 4096) return BQO_ERR_ARG;
     if (fegetround() != FE_TONEAREST) return BQO_ERR_ARG;
@@ -210,8 +272,10 @@ int bqo_quantize_scheme(const uint16_t *W, int wtype, int64_t rows, int64_t cols
             for (int i = 0; i < group; ++i) buf[i] = decode(src[i], wtype);
             float s;
             int z;
-            int rc = scheme ? bqo_quantize_group_sym(buf, group, bits, &s, &z, codes + n * cols + j * group)
-                            : bqo_quantize_group(buf, group, bits, &s, &z, codes + n * cols + j * group);
+            uint8_t *q = codes + n * cols + j * group;
+            int rc = scheme == 1 ? bqo_quantize_group_sym(buf, group, bits, &s, &z, q)
+                   : scheme == 2 ? bqo_quantize_group_s16(buf, group, bits, &s, &z, q)
+                                 : bqo_quantize_group(buf, group, bits, &s, &z, q);
             if (rc) return rc;
             scales[n * G + j] = s;
             zeros[n * G + j] = (uint8_t)z;

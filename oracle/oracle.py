@@ -58,6 +58,10 @@ def lib():
             L.bqo_quantize_scheme.restype = i32
             L.bqo_quantize_group_sym.argtypes = [vp, i32, i32, vp, vp, vp]
             L.bqo_quantize_group_sym.restype = i32
+            L.bqo_quantize_group_s16.argtypes = [vp, i32, i32, vp, vp, vp]
+            L.bqo_quantize_group_s16.restype = i32
+            L.bqo_f32_to_f16.argtypes = [ctypes.c_float]
+            L.bqo_f32_to_f16.restype = ctypes.c_uint16
             L.bqo_code_position.argtypes = [i32, i64, i64, i64, i64, i32, vp, vp]
             L.bqo_code_position.restype = None
             L.bqo_pack.argtypes = [vp, i64, i64, i32, i32, vp]
@@ -144,14 +148,22 @@ def quantize_group(x: np.ndarray, bits: int, scheme: str = "asymmetric"):
     q = np.zeros(x.size, dtype=np.uint8)
     s = ctypes.c_float()
     z = ctypes.c_int()
-    fn = lib().bqo_quantize_group_sym if scheme == "symmetric" else lib().bqo_quantize_group
+    fn = {"symmetric": lib().bqo_quantize_group_sym,
+          "asymmetric_f16_scale": lib().bqo_quantize_group_s16}.get(scheme, lib().bqo_quantize_group)
     rc = fn(_p(x), x.size, bits, ctypes.byref(s), ctypes.byref(z), _p(q))
     if rc:
         raise OracleError(f"bqo_quantize_group rc={rc}")
     return float(np.float32(s.value)), int(z.value), q
 
 
-SCHEMES = {"asymmetric": 0, "symmetric": 1}
+def f32_to_f16_bits(values) -> np.ndarray:
+    """binary32 values -> binary16 bit patterns (round to nearest, ties to even)."""
+    v = np.ascontiguousarray(values, dtype=np.float32).ravel()
+    L = lib()
+    return np.array([L.bqo_f32_to_f16(float(a)) for a in v], dtype=np.uint16).reshape(np.shape(values))
+
+
+SCHEMES = {"asymmetric": 0, "symmetric": 1, "asymmetric_f16_scale": 2}
 
 
 def quantize(w_bits: np.ndarray, wtype: str, bits: int, group: int, threads: int = 1, scheme: str = "asymmetric"):

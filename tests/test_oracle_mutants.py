@@ -49,6 +49,9 @@ MUTANTS = {
                                   "            int64_t j = k % G;\n            float d"),
     "dequant64_zero_sign": ("out[n * cols + k] = (double)((int)codes[n * cols + k] - (int)zeros[n * G + j])",
                             "out[n * cols + k] = (double)((int)codes[n * cols + k] + (int)zeros[n * G + j])"),
+    "f16_scale_not_rounded": ("        s = bqo_f16_to_f32(bqo_f32_to_f16(s));\n", ""),
+    "f16_round_half_away": ("    float n = nearbyintf(ldexpf(a, -ulp_exp));", "    float n = roundf(ldexpf(a, -ulp_exp));"),
+    "f16_subnormal_step": ("    if (ulp_exp < -24) ulp_exp = -24;", "    if (ulp_exp < -25) ulp_exp = -25;"),
     "dequant64_scale_transposed": ("                                * (double)scales[n * G + j];\n        }\n}",
                                    "                                * (double)scales[j * rows + n];\n        }\n}"),
 }
@@ -75,6 +78,9 @@ PINS = [
     (P.test_sym_page_scale_example, {}),
     (P.test_grad_input_closed_form, {"bits": 4, "g": 128}),
     (P.test_grad_input_adjoint, {"bits": 4, "g": 32}),
+    (P.test_f16_scale_worked_example, {}),
+    (P.test_f32_to_f16_matches_library_rounding, {}),
+    (P.test_f16_scale_exact_rational_arithmetic, {}),
 ]
 
 

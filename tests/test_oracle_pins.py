@@ -627,3 +627,78 @@ def test_sym_matrix_matches_groups():
         for j in range(4):
             s, z, q = O.quantize_group(W[n, 64 * j:64 * (j + 1)].astype(np.float32), 4, scheme="symmetric")
             assert scales[n, j] == s and zeros[n, j] == z and (codes[n, 64 * j:64 * (j + 1)] == q).all()
+
+
+# --------------------------------------------------------------------------
+# binary16 group scales (the fp16-scale format variant)
+# --------------------------------------------------------------------------
+
+def test_f16_scale_worked_example():
+    g = read_golden("int4_f16scale_worked.txt")
+    x = np.array([float(v) for v in g["x"]], dtype=np.float32)
+    s, z, q = O.quantize_group(x, int(g["bits"][0]), "asymmetric_f16_scale")
+    assert s == float(g["s"][0])
+    assert int(O.f32_to_f16_bits(np.float32(s))) == int(g["s_f16_bits"][0], 16)
+    assert z == int(g["z"][0])
+    assert q.tolist() == [int(v) for v in g["q"]]
+
+
+def test_f32_to_f16_matches_library_rounding():
+    """The oracle's binary16 rounding against numpy's (IEEE round to nearest,
+    ties to even): every binary16 value and its neighbours, the midpoints
+    between consecutive binary16 values (ties), the subnormal range, the
+    overflow boundary and random magnitudes over the whole range."""
+    rng = np.random.default_rng(7)
+    h = np.arange(0, 0x7C00, dtype=np.uint16)
+    exact = h.view(np.float16).astype(np.float32)
+    up = np.nextafter(exact, np.float32(np.inf))
+    down = np.nextafter(exact, np.float32(0))
+    mids = ((exact[:-1].astype(np.float64) + exact[1:].astype(np.float64)) / 2).astype(np.float32)
+    edge = np.array([0.0, -0.0, 65504.0, 65519.99, 65520.0, 65536.0, 1e10, 2.0 ** -24, 2.0 ** -25,
+                     2.0 ** -25 * 1.0001, 2.0 ** -26, 1e-10, 6.1e-5], dtype=np.float32)
+    rnd = (rng.uniform(-30, 17, 20000).astype(np.float64))
+    rnd = (np.sign(rng.normal(size=rnd.size)) * 2.0 ** rnd).astype(np.float32)
+    vals = np.concatenate([exact, up, down[1:], mids, edge, -mids[::97], rnd])
+    got = O.f32_to_f16_bits(vals)
+    with np.errstate(over="ignore"):  # the overflow cases are intended (-> infinity)
+        want = vals.astype(np.float16).view(np.uint16)
+    bad = np.nonzero(got != want)[0]
+    assert bad.size == 0, (vals[bad[:5]], got[bad[:5]], want[bad[:5]])
+
+
+def exact_group_f16_scale(x32: np.ndarray, bits: int):
+    """R1-R3 in exact rational arithmetic, with the scale rounded to binary16
+    by numpy (round to nearest, ties to even) and used for z and the codes."""
+    qmax = (1 << bits) - 1
+    xs = [Fraction(float(v)) for v in x32]
+    lo = min(min(xs), Fraction(0))
+    hi = max(max(xs), Fraction(0))
+    s32 = rne_f32(rne_f32(hi - lo) / qmax)
+    if s32 == 0:
+        return 0.0, 0, [0] * len(xs)
+    s16 = Fraction(float(np.float16(float(s32))))
+    if s16 == 0:
+        s16 = Fraction(1, 2 ** 24)
+    z = rne_int(rne_f32(-lo / s16))
+    q = [min(max(rne_int(rne_f32(v / s16)) + z, 0), qmax) for v in xs]
+    return float(s16), z, q
+
+
+def test_f16_scale_exact_rational_arithmetic():
+    rng = np.random.default_rng(123)
+    groups = [g.astype(np.float16).astype(np.float32) for g in _random_groups(rng, 120, 16)]
+    # tiny groups whose scale falls into (or below) the binary16 subnormals
+    for e in (-18, -22, -26, -30):
+        groups.append((rng.normal(0, 2.0 ** e, 16)).astype(np.float16).astype(np.float32))
+    # near ties of x / s16
+    for _ in range(150):
+        base = rng.normal(0, 1, 16).astype(np.float16).astype(np.float32)
+        s16 = float(np.float16((float(base.max()) - min(float(base.min()), 0.0)) / 15))
+        k = int(rng.integers(-7, 8))
+        base[4] = np.float32(np.float16((k + 0.5) * s16))
+        groups.append(base)
+    for i, x in enumerate(groups):
+        for bits in (2, 4):
+            s, z, q = O.quantize_group(x, bits, "asymmetric_f16_scale")
+            es, ez, eq = exact_group_f16_scale(x, bits)
+            assert (s, z, q.tolist()) == (es, ez, eq), (i, bits)
