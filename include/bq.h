@@ -184,6 +184,25 @@ bq_status bq_quantize_symmetric(const void *W, bq_dtype wtype, int64_t rows, int
                                 bq_layout layout, void *packed, float *scales, uint8_t *zeros, void *stream);
 
 /*
+ * bq_quantize_f16s: the asymmetric MinMax scheme of bq_quantize with the
+ * group scales stored as binary16 -- a storage format that cuts the
+ * metadata from 5 to 3 bytes per group (INT2 g64: from 24% to 16% of the
+ * linear layer's bytes).  s is computed as in bq_quantize, rounded to the
+ * nearest binary16 (ties to even; a positive s below the binary16 range
+ * becomes 2^-24, one above it sets BQ_ERR_NONFINITE), and z and the codes
+ * are then computed from that stored s16 with bq_quantize's steps, so
+ * dequant(q) = (q - z) * s16 ("大模型量化实战", section 2.2 formulas; "低比特
+ * 量化", Zero Point).  A code that round(x / s16) + z pushes past 2^b - 1
+ * is clamped.  Only the linear layer's pairs: bits 4 with group 128, bits 2
+ * with group 64 (others BQ_ERR_UNSUPPORTED).
+ *   scales   binary16 bit patterns, same count and order as bq_quantize's
+ *            fp32 scales, 2-byte aligned (16-byte for bq_linear_f16s)
+ * Other arguments, layouts, outputs and errors as bq_quantize.
+ */
+bq_status bq_quantize_f16s(const void *W, bq_dtype wtype, int64_t rows, int64_t cols, int bits, int group,
+                           bq_layout layout, void *packed, uint16_t *scales, uint8_t *zeros, void *stream);
+
+/*
  * bq_fake_quantize: W_out = dequant(quant(W)) in one pass, without storing
  * codes, scales or zeros -- the forward of quantization-aware training
  * ("大模型量化实战", section 5.2: a FakeQuantize module simulates
@@ -222,6 +241,17 @@ bq_status bq_linear(const void *x, bq_dtype xtype, int64_t M, int64_t K,
                     const void *packed, const float *scales, const uint8_t *zeros,
                     const uint8_t *bit_map, int bits, int group, int64_t N,
                     bq_layout layout, void *y, void *stream);
+
+/*
+ * bq_linear_f16s: bq_linear for weights from bq_quantize_f16s (binary16
+ * scales, uniform width, bits 4 with group 128 or bits 2 with group 64; no
+ * bit map).  The binary16 scale is exact in fp32, so the products are
+ * those of bq_linear with the same scale values.  Arguments, shape rules,
+ * alignment and errors as bq_linear.
+ */
+bq_status bq_linear_f16s(const void *x, bq_dtype xtype, int64_t M, int64_t K,
+                         const void *packed, const uint16_t *scales, const uint8_t *zeros,
+                         int bits, int group, int64_t N, bq_layout layout, void *y, void *stream);
 
 /*
  * bq_linear_grad_input: dx[M, K] = dy[M, N] . dequant(W), the gradient of

@@ -34,7 +34,7 @@ EXPORTS = (
     "bq_packed_bytes", "bq_group_count", "bq_mixed_offsets", "bq_quantize", "bq_quantize_symmetric",
     "bq_quantize_mixed",
     "bq_dequantize", "bq_fake_quantize", "bq_linear", "bq_linear_grad_input", "bq_check_division",
-    "bq_check_const_division",
+    "bq_check_const_division", "bq_quantize_f16s", "bq_linear_f16s",
     "bq_selftest_bounded_wait", "bq_set_option", "bq_get_option", "bq_device_status",
     "bq_status_string", "bq_version",
 )
@@ -71,6 +71,8 @@ def lib(path: str | None = None):
     L.bq_quantize.restype = i32
     L.bq_quantize_symmetric.argtypes = [vp, i32, i64, i64, i32, i32, i32, vp, vp, vp, vp]
     L.bq_quantize_symmetric.restype = i32
+    L.bq_quantize_f16s.argtypes = [vp, i32, i64, i64, i32, i32, i32, vp, vp, vp, vp]
+    L.bq_quantize_f16s.restype = i32
     L.bq_quantize_mixed.argtypes = [vp, i32, i64, i64, vp, i32, vp, vp, vp, vp]
     L.bq_quantize_mixed.restype = i32
     L.bq_dequantize.argtypes = [vp, vp, vp, vp, i32, i32, i64, i64, i32, vp, i32, vp]
@@ -79,6 +81,8 @@ def lib(path: str | None = None):
     L.bq_fake_quantize.restype = i32
     L.bq_linear.argtypes = [vp, i32, i64, i64, vp, vp, vp, vp, i32, i32, i64, i32, vp, vp]
     L.bq_linear.restype = i32
+    L.bq_linear_f16s.argtypes = [vp, i32, i64, i64, vp, vp, vp, i32, i32, i64, i32, vp, vp]
+    L.bq_linear_f16s.restype = i32
     L.bq_linear_grad_input.argtypes = [vp, i32, i64, i64, vp, vp, vp, vp, i32, i32, i64, i32, vp, vp]
     L.bq_linear_grad_input.restype = i32
     L.bq_check_division.argtypes = [ctypes.c_uint32, ctypes.c_uint32, i32, vp, vp]
@@ -149,19 +153,22 @@ def bq_mixed_offsets(bit_map, rows: int, cols: int):
 
 def bq_quantize(W: torch.Tensor, bits: int, group: int | None = None, layout: str = "interleaved",
                 out=None, stream=None, scheme: str = "asymmetric"):
-    """Quantize W [N, K] (fp16/bf16, CUDA) with the asymmetric MinMax scheme (default) or the
-    symmetric abs-max one.  Returns (packed u8, scales f32, zeros u8): scales / zeros are [N, K/g]
-    in the canonical layout and flat (128-row-block-major order) in the interleaved one."""
+    """Quantize W [N, K] (fp16/bf16, CUDA) with the asymmetric MinMax scheme (default), the
+    symmetric abs-max one, or the MinMax scheme with binary16 scales ("asymmetric_f16_scale").
+    Returns (packed u8, scales, zeros u8): scales f32 (f16 for the binary16 format) / zeros are
+    [N, K/g] in the canonical layout and flat (128-row-block-major order) in the interleaved one."""
     group = group or GROUP_OF_BITS[bits]
     N, K = W.shape
+    s16 = scheme == "asymmetric_f16_scale"
     if out is None:
         packed = torch.empty(max(1, bq_packed_bytes(N, K, bits)), dtype=torch.uint8, device=W.device)
         mshape = (N, K // group) if layout == "canonical" else (N * (K // group),)
-        scales = torch.empty(mshape, dtype=torch.float32, device=W.device)
+        scales = torch.empty(mshape, dtype=torch.float16 if s16 else torch.float32, device=W.device)
         zeros = torch.empty(mshape, dtype=torch.uint8, device=W.device)
     else:
         packed, scales, zeros = out
-    fn = lib().bq_quantize_symmetric if scheme == "symmetric" else lib().bq_quantize
+    fn = {"symmetric": lib().bq_quantize_symmetric, "asymmetric_f16_scale": lib().bq_quantize_f16s,
+          "asymmetric": lib().bq_quantize}[scheme]
     st = fn(_ptr(W), DTYPE_CODE[W.dtype], N, K, bits, group, LAYOUTS[layout],
             _ptr(packed), _ptr(scales), _ptr(zeros), _stream(stream))
     _check("bq_quantize", st)
@@ -211,10 +218,18 @@ def bq_fake_quantize(W: torch.Tensor, bits: int, group: int | None = None, out_d
 
 def bq_linear(x: torch.Tensor, packed, scales, zeros, N: int, bits: int = 4, group: int | None = None,
               bit_map_dev=None, layout: str = "interleaved", out=None, stream=None):
-    """y [M, N] = x [M, K] . dequant(W)^T, y in x's dtype."""
+    """y [M, N] = x [M, K] . dequant(W)^T, y in x's dtype.  fp16 `scales` (from the binary16
+    scale format) select bq_linear_f16s."""
     group = group or GROUP_OF_BITS.get(bits, 0)
     M, K = x.shape
     y = out if out is not None else torch.empty((M, N), dtype=x.dtype, device=x.device)
+    if scales.dtype == torch.float16:
+        if bit_map_dev is not None:
+            raise ValueError("binary16 scales take no width map")
+        st = lib().bq_linear_f16s(_ptr(x), DTYPE_CODE[x.dtype], M, K, _ptr(packed), _ptr(scales), _ptr(zeros),
+                                  bits, group, N, LAYOUTS[layout], _ptr(y), _stream(stream))
+        _check("bq_linear_f16s", st)
+        return y
     st = lib().bq_linear(_ptr(x), DTYPE_CODE[x.dtype], M, K, _ptr(packed), _ptr(scales), _ptr(zeros),
                          _ptr(bit_map_dev), bits, group, N, LAYOUTS[layout], _ptr(y), _stream(stream))
     _check("bq_linear", st)

@@ -118,16 +118,23 @@ int tile_width(int bits) { return bits == 4 ? 64 : 128; }
 // ---------------------------------------------------------------------------
 
 template <int WT, int BITS, int SCHEME>
-bq_status quantize_canonical(const uint16_t *W, int64_t elems, int group, uint8_t *packed, float *scales,
+bq_status quantize_canonical(const uint16_t *W, int64_t elems, int group, uint8_t *packed, void *scales,
                              uint8_t *zeros, cudaStream_t st) {
   const int64_t grid = grid_for((elems + 255) / 256);
 #define BQ_QC(G)                                                                              \
   case G:                                                                                     \
     quantize_canonical_kernel<WT, BITS, G, 4, SCHEME><<<grid, kThreads, 0, st>>>(W, elems, packed, scales, zeros); \
     break;
-  switch (group) {
-    BQ_QC(8) BQ_QC(16) BQ_QC(32) BQ_QC(64) BQ_QC(128) BQ_QC(256)
-    default: return BQ_ERR_UNSUPPORTED;
+  if constexpr (SCHEME == 2) {  // binary16 scales: the linear layer's groups, INT4 g128 and INT2 g64
+    switch (group) {
+      BQ_QC(64) BQ_QC(128)
+      default: return BQ_ERR_UNSUPPORTED;
+    }
+  } else {
+    switch (group) {
+      BQ_QC(8) BQ_QC(16) BQ_QC(32) BQ_QC(64) BQ_QC(128) BQ_QC(256)
+      default: return BQ_ERR_UNSUPPORTED;
+    }
   }
 #undef BQ_QC
   return launch_status();
@@ -136,7 +143,7 @@ bq_status quantize_canonical(const uint16_t *W, int64_t elems, int group, uint8_
 // Interleaved layout: the TMA-staged kernel, two CTAs per SM, each with a ring
 // of super-units (64 rows x U columns) in about 110 KB of shared memory.
 template <int WT, int BITS, int G, int SCHEME>
-bq_status quantize_tma(const uint16_t *W, int64_t N, int64_t K, uint8_t *packed, float *scales, uint8_t *zeros,
+bq_status quantize_tma(const uint16_t *W, int64_t N, int64_t K, uint8_t *packed, void *scales, uint8_t *zeros,
                        cudaStream_t st) {
   constexpr int U = UnitGeom<BITS, G>::U;
   constexpr int SU = (U / 64) * 8192;
@@ -157,9 +164,13 @@ bq_status quantize_tma(const uint16_t *W, int64_t N, int64_t K, uint8_t *packed,
 }
 
 template <int WT, int BITS, int SCHEME>
-bq_status quantize_tiled(const uint16_t *W, int64_t N, int64_t K, int group, uint8_t *packed, float *scales,
+bq_status quantize_tiled(const uint16_t *W, int64_t N, int64_t K, int group, uint8_t *packed, void *scales,
                          uint8_t *zeros, cudaStream_t st) {
-  switch (group) {
+  if constexpr (SCHEME == 2) {  // binary16 scales: the linear layer's groups, INT4 g128 and INT2 g64
+    if (group == 64) return quantize_tma<WT, BITS, 64, SCHEME>(W, N, K, packed, scales, zeros, st);
+    if (group == 128) return quantize_tma<WT, BITS, 128, SCHEME>(W, N, K, packed, scales, zeros, st);
+    return BQ_ERR_UNSUPPORTED;
+  } else switch (group) {
     case 16: return quantize_tma<WT, BITS, 16, SCHEME>(W, N, K, packed, scales, zeros, st);
     case 32: return quantize_tma<WT, BITS, 32, SCHEME>(W, N, K, packed, scales, zeros, st);
     case 64: return quantize_tma<WT, BITS, 64, SCHEME>(W, N, K, packed, scales, zeros, st);
@@ -303,10 +314,10 @@ GemvGeom gemv_geometry(int M, int64_t N, int64_t K, int SC, int G_min) {
   return g;
 }
 
-template <int XT, int BITS, int G, int NB, bool MIXED>
+template <int XT, int BITS, int G, int NB, bool MIXED, bool S16>
 bq_status launch_gemv_t(const GemvGeom &g, GemvArgs a, int G_min, cudaStream_t st) {
-  auto kern = gemv_kernel<XT, BITS, G, NB, MIXED>;
-  if (!ensure_smem<gemv_kernel<XT, BITS, G, NB, MIXED>>(kMaxSmem)) return BQ_ERR_CUDA;
+  auto kern = gemv_kernel<XT, BITS, G, NB, MIXED, S16>;
+  if (!ensure_smem<gemv_kernel<XT, BITS, G, NB, MIXED, S16>>(kMaxSmem)) return BQ_ERR_CUDA;
   a.stages = g.stages;
   a.KC = g.KC;
   a.L = gemv_smem_layout(a.M, 8 * NB, g.KC, (int)(g.KC / G_min), g.stages);
@@ -342,18 +353,19 @@ bq_status launch_gemv_t(const GemvGeom &g, GemvArgs a, int G_min, cudaStream_t s
 
 // Stage width: 256 columns at 4 bits, 512 at 2 bits; a mixed matrix uses
 // 512-column splits so that both widths tile every CTA's slice.
-template <int XT, int BITS, int G, bool MIXED>
+template <int XT, int BITS, int G, bool MIXED, bool S16 = false>
 bq_status launch_gemv_dispatch(const GemvArgs &a, cudaStream_t st) {
   const int split_unit = MIXED ? 512 : StageG<BITS, G>::SC;
   if (a.K % split_unit) return BQ_ERR_SHAPE;
   const int G_min = MIXED ? 64 : G;
   GemvGeom g = gemv_geometry(a.M, a.N, a.K, split_unit, G_min);
-  if (g.NB == 1) return launch_gemv_t<XT, BITS, G, 1, MIXED>(g, a, G_min, st);
-  return launch_gemv_t<XT, BITS, G, 2, MIXED>(g, a, G_min, st);
+  if (g.NB == 1) return launch_gemv_t<XT, BITS, G, 1, MIXED, S16>(g, a, G_min, st);
+  return launch_gemv_t<XT, BITS, G, 2, MIXED, S16>(g, a, G_min, st);
 }
 
+// s16: binary16 scales (uniform INT4 g128 or INT2 g64 only).
 template <int XT>
-bq_status gemv_dispatch(const uint16_t *x, int M, int64_t K, const uint8_t *packed, const float *scales,
+bq_status gemv_dispatch(const uint16_t *x, int M, int64_t K, const uint8_t *packed, const void *scales, bool s16,
                         const uint8_t *zeros, const uint8_t *bit_map, int bits, int group, int64_t N, uint16_t *y,
                         cudaStream_t st) {
   GemvArgs a = {};
@@ -366,6 +378,12 @@ bq_status gemv_dispatch(const uint16_t *x, int M, int64_t K, const uint8_t *pack
   a.K = K;
   a.N = N;
   a.M = M;
+  if (s16) {
+    if (bit_map) return BQ_ERR_UNSUPPORTED;
+    if (bits == 4 && group == 128) return launch_gemv_dispatch<XT, 4, 128, false, true>(a, st);
+    if (bits == 2 && group == 64) return launch_gemv_dispatch<XT, 2, 64, false, true>(a, st);
+    return BQ_ERR_UNSUPPORTED;
+  }
   if (bit_map) return launch_gemv_dispatch<XT, 4, 128, true>(a, st);
 #define BQ_GV(B, G_) \
   if (bits == B && group == G_) return launch_gemv_dispatch<XT, B, G_, false>(a, st);
@@ -476,9 +494,9 @@ bool make_x_map(CUtensorMap *map, const uint16_t *x, int64_t M, int64_t K, int x
   return make_map_2d(map, x, M, K, xt == 1, 64, kGemmTokTile);
 }
 
-template <int XT, int BITS, int G, bool MIXED = false>
+template <int XT, int BITS, int G, bool MIXED = false, bool S16 = false>
 bq_status launch_gemm_t(const uint16_t *x, int64_t M, int64_t K, const GemmArgs &a, cudaStream_t st) {
-  auto kern = gemm_kernel<XT, BITS, G, MIXED>;
+  auto kern = gemm_kernel<XT, BITS, G, MIXED, S16>;
   // the warpgroups' setmaxnreg shares must fit in the registers the block is
   // launched with, or the raising warpgroups would wait forever (a property
   // of the compiled kernel, checked once per process)
@@ -489,7 +507,7 @@ bq_status launch_gemm_t(const uint16_t *x, int64_t M, int64_t K, const GemmArgs 
     regs_ok.store((int64_t)fa.numRegs * kGemmThreads >= (int64_t)kGemmRegsNeeded ? 1 : -1, std::memory_order_release);
   }
   if (regs_ok.load(std::memory_order_acquire) < 0) return BQ_ERR_UNSUPPORTED;
-  if (!ensure_smem<gemm_kernel<XT, BITS, G, MIXED>>(GemmSmem::total)) return BQ_ERR_CUDA;
+  if (!ensure_smem<gemm_kernel<XT, BITS, G, MIXED, S16>>(GemmSmem::total)) return BQ_ERR_CUDA;
   CUtensorMap map;
   if (!make_x_map(&map, x, M, K, XT)) return BQ_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
@@ -522,7 +540,7 @@ bool gemm_eligible(int64_t M, int64_t N, const uint8_t *bit_map, int group) {
 }
 
 template <int XT>
-bq_status gemm_dispatch(const uint16_t *x, int64_t M, int64_t K, const uint8_t *packed, const float *scales,
+bq_status gemm_dispatch(const uint16_t *x, int64_t M, int64_t K, const uint8_t *packed, const void *scales, bool s16,
                         const uint8_t *zeros, const uint8_t *bit_map, int bits, int group, int64_t N, uint16_t *y,
                         cudaStream_t st) {
   GemmArgs a = {};
@@ -534,6 +552,12 @@ bq_status gemm_dispatch(const uint16_t *x, int64_t M, int64_t K, const uint8_t *
   a.M = M;
   a.K = K;
   a.N = N;
+  if (s16) {
+    if (bit_map) return BQ_ERR_UNSUPPORTED;
+    if (bits == 4 && group == 128) return launch_gemm_t<XT, 4, 128, false, true>(x, M, K, a, st);
+    if (bits == 2 && group == 64) return launch_gemm_t<XT, 2, 64, false, true>(x, M, K, a, st);
+    return BQ_ERR_UNSUPPORTED;
+  }
   if (bit_map) return launch_gemm_t<XT, 4, 128, true>(x, M, K, a, st);
 #define BQ_GM(B, G_) \
   if (bits == B && group == G_) return launch_gemm_t<XT, B, G_>(x, M, K, a, st);
@@ -547,11 +571,12 @@ bool linear_group_ok(int bits, int g) {
   return g == 32 || g == 64 || g == 128 || g == 256;
 }
 
-// bq_quantize / bq_quantize_symmetric: the same validation and layouts,
-// SCHEME 0 asymmetric MinMax, 1 symmetric abs-max.
+// bq_quantize / bq_quantize_symmetric / bq_quantize_f16s: the same
+// validation and layouts, SCHEME 0 asymmetric MinMax, 1 symmetric abs-max,
+// 2 asymmetric MinMax with binary16 scales.
 template <int SCHEME>
 bq_status quantize_any(const void *W, bq_dtype wtype, int64_t rows, int64_t cols, int bits, int group,
-                       bq_layout layout, void *packed, float *scales, uint8_t *zeros, void *stream) {
+                       bq_layout layout, void *packed, void *scales, uint8_t *zeros, void *stream) {
   if (rows < 0 || cols < 0) return BQ_ERR_SHAPE;
   if (!valid_bits(bits) || (wtype != BQ_F16 && wtype != BQ_BF16)) return BQ_ERR_UNSUPPORTED;
   if (layout != BQ_LAYOUT_CANONICAL && layout != BQ_LAYOUT_INTERLEAVED) return BQ_ERR_UNSUPPORTED;
@@ -565,7 +590,7 @@ bq_status quantize_any(const void *W, bq_dtype wtype, int64_t rows, int64_t cols
   }
   if (rows == 0 || cols == 0) return BQ_OK;
   if (!W || !packed || !scales || !zeros) return BQ_ERR_NULL;
-  if (!aligned(W, 16) || !aligned(packed, 16) || !aligned(scales, 4)) return BQ_ERR_ALIGN;
+  if (!aligned(W, 16) || !aligned(packed, 16) || !aligned(scales, SCHEME == 2 ? 2 : 4)) return BQ_ERR_ALIGN;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const uint16_t *w = reinterpret_cast<const uint16_t *>(W);
   uint8_t *pk = reinterpret_cast<uint8_t *>(packed);
@@ -643,6 +668,12 @@ bq_status bq_quantize(const void *W, bq_dtype wtype, int64_t rows, int64_t cols,
 bq_status bq_quantize_symmetric(const void *W, bq_dtype wtype, int64_t rows, int64_t cols, int bits, int group,
                                 bq_layout layout, void *packed, float *scales, uint8_t *zeros, void *stream) {
   return quantize_any<1>(W, wtype, rows, cols, bits, group, layout, packed, scales, zeros, stream);
+}
+
+bq_status bq_quantize_f16s(const void *W, bq_dtype wtype, int64_t rows, int64_t cols, int bits, int group,
+                           bq_layout layout, void *packed, uint16_t *scales, uint8_t *zeros, void *stream) {
+  if (!((bits == 4 && group == 128) || (bits == 2 && group == 64))) return BQ_ERR_UNSUPPORTED;
+  return quantize_any<2>(W, wtype, rows, cols, bits, group, layout, packed, scales, zeros, stream);
 }
 
 bq_status bq_quantize_mixed(const void *W, bq_dtype wtype, int64_t rows, int64_t cols, const uint8_t *bit_map,
@@ -725,10 +756,16 @@ bq_status bq_fake_quantize(const void *W, bq_dtype wtype, int64_t rows, int64_t 
   return fake_quant_bits<1, 2>(w, elems, bits, group, W_out, st);
 }
 
-bq_status bq_linear(const void *x, bq_dtype xtype, int64_t M, int64_t K, const void *packed, const float *scales,
-                    const uint8_t *zeros, const uint8_t *bit_map, int bits, int group, int64_t N,
-                    bq_layout layout, void *y, void *stream) {
+}  // extern "C"
+
+namespace {
+
+// bq_linear and bq_linear_f16s: s16 selects binary16 scales.
+bq_status linear_any(const void *x, bq_dtype xtype, int64_t M, int64_t K, const void *packed, const void *scales,
+                     bool s16, const uint8_t *zeros, const uint8_t *bit_map, int bits, int group, int64_t N,
+                     bq_layout layout, void *y, void *stream) {
   if (M < 0 || K < 0 || N < 0) return BQ_ERR_SHAPE;
+  if (s16 && (bit_map || !((bits == 4 && group == 128) || (bits == 2 && group == 64)))) return BQ_ERR_UNSUPPORTED;
   if (xtype != BQ_F16 && xtype != BQ_BF16) return BQ_ERR_UNSUPPORTED;
   if (layout != BQ_LAYOUT_INTERLEAVED) return BQ_ERR_UNSUPPORTED;
   if (bit_map) {
@@ -751,17 +788,35 @@ bq_status bq_linear(const void *x, bq_dtype xtype, int64_t M, int64_t K, const v
   uint16_t *yy = reinterpret_cast<uint16_t *>(y);
   const uint8_t *pk = reinterpret_cast<const uint8_t *>(packed);
   if (gemm_eligible(M, N, bit_map, group))
-    return (xtype == BQ_BF16) ? gemm_dispatch<1>(xx, M, K, pk, scales, zeros, bit_map, bits, group, N, yy, st)
-                              : gemm_dispatch<0>(xx, M, K, pk, scales, zeros, bit_map, bits, group, N, yy, st);
+    return (xtype == BQ_BF16) ? gemm_dispatch<1>(xx, M, K, pk, scales, s16, zeros, bit_map, bits, group, N, yy, st)
+                              : gemm_dispatch<0>(xx, M, K, pk, scales, s16, zeros, bit_map, bits, group, N, yy, st);
   // Otherwise token blocks of at most 16 go through the decode kernel.
   for (int64_t m0 = 0; m0 < M; m0 += 16) {
     const int mb = (int)((M - m0) < 16 ? (M - m0) : 16);
     bq_status s = (xtype == BQ_BF16)
-                      ? gemv_dispatch<1>(xx + m0 * K, mb, K, pk, scales, zeros, bit_map, bits, group, N, yy + m0 * N, st)
-                      : gemv_dispatch<0>(xx + m0 * K, mb, K, pk, scales, zeros, bit_map, bits, group, N, yy + m0 * N, st);
+                      ? gemv_dispatch<1>(xx + m0 * K, mb, K, pk, scales, s16, zeros, bit_map, bits, group, N,
+                                         yy + m0 * N, st)
+                      : gemv_dispatch<0>(xx + m0 * K, mb, K, pk, scales, s16, zeros, bit_map, bits, group, N,
+                                         yy + m0 * N, st);
     if (s != BQ_OK) return s;
   }
   return BQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+bq_status bq_linear(const void *x, bq_dtype xtype, int64_t M, int64_t K, const void *packed, const float *scales,
+                    const uint8_t *zeros, const uint8_t *bit_map, int bits, int group, int64_t N,
+                    bq_layout layout, void *y, void *stream) {
+  return linear_any(x, xtype, M, K, packed, scales, false, zeros, bit_map, bits, group, N, layout, y, stream);
+}
+
+bq_status bq_linear_f16s(const void *x, bq_dtype xtype, int64_t M, int64_t K, const void *packed,
+                         const uint16_t *scales, const uint8_t *zeros, int bits, int group, int64_t N,
+                         bq_layout layout, void *y, void *stream) {
+  return linear_any(x, xtype, M, K, packed, scales, true, zeros, nullptr, bits, group, N, layout, y, stream);
 }
 
 bq_status bq_linear_grad_input(const void *dy, bq_dtype dtype, int64_t M, int64_t N, const void *packed,

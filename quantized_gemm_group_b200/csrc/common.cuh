@@ -194,7 +194,11 @@ BQ_DEV GroupParams group_params_sym(float mn, float mx) {
   return p;
 }
 
-// SCHEME 0: asymmetric MinMax (below); 1: symmetric abs-max.
+// SCHEME 0: asymmetric MinMax (below); 1: symmetric abs-max; 2: asymmetric
+// MinMax with the scale stored as binary16: s rounded to the nearest binary16
+// (ties to even; a positive s below the binary16 range takes 2^-24, one
+// above it marks the group non-finite), and z and the codes computed from
+// that stored value.
 template <int QMAX, int SCHEME = 0>
 BQ_DEV GroupParams group_params(float mn, float mx) {
   if (SCHEME == 1) return group_params_sym<QMAX>(mn, mx);
@@ -203,6 +207,10 @@ BQ_DEV GroupParams group_params(float mn, float mx) {
   float lo = fminf(mn, 0.0f);
   float hi = fmaxf(mx, 0.0f);
   float s = div_const<QMAX>(__fsub_rn(hi, lo));
+  if (SCHEME == 2 && s > 0.0f && s <= 3.402823466e38f) {
+    s = __half2float(__float2half_rn(s));
+    if (s == 0.0f) s = 0x1p-24f;
+  }
   p.bad |= !(s <= 3.402823466e38f);
   if (p.bad || s == 0.0f) {
     // all-zero group: s = 0, z = 0 and every x is +-0, so x / 1 rounds to 0
@@ -245,6 +253,13 @@ BQ_DEV float2 rounded_quotients(float2 v, const GroupParams &p) {
     t = make_float2(__fdiv_rn(v.x, p.sd), __fdiv_rn(v.y, p.sd));
   }
   return __fadd2_rn(t, make_float2(kRoundMagic, kRoundMagic));
+}
+
+// Store a group scale: fp32, or (SCHEME 2) the binary16 value it already is.
+template <int SCHEME>
+BQ_DEV void store_scale(void *scales, int64_t i, float s) {
+  if (SCHEME == 2) reinterpret_cast<uint16_t *>(scales)[i] = __half_as_ushort(__float2half_rn(s));
+  else reinterpret_cast<float *>(scales)[i] = s;
 }
 
 // Codes of two elements of one group.

@@ -99,7 +99,7 @@ struct GemmSmem {
 
 struct GemmArgs {
   const uint8_t *packed;
-  const float *scales;
+  const void *scales;  // fp32, or binary16 when the kernel's S16 is set
   const uint8_t *zeros;
   const uint8_t *bit_map;
   uint16_t *y;
@@ -409,8 +409,16 @@ BQ_DEV void gemm_mma(const GemmArgs &a, int which, uint32_t tmem, uint32_t sbase
 
 // Epilogue warp e (0..15, warps 8-23): TMEM lanes 32 (warp % 4) .. +31 (weight rows),
 // token columns 64 (e / 4) .. +63.
-template <int XT, int BITS, int G>
-BQ_DEV void gemm_epilogue(const GemmArgs &a, const float *sc, int e, int warp, int lane, uint32_t tmem,
+// One group scale from the block-major metadata: fp32, or binary16 (exact
+// in fp32).
+template <bool S16>
+BQ_DEV float load_scale(const void *sc, int64_t i) {
+  if (S16) return __half2float(__ushort_as_half(__ldg(reinterpret_cast<const unsigned short *>(sc) + i)));
+  return __ldg(reinterpret_cast<const float *>(sc) + i);
+}
+
+template <int XT, int BITS, int G, bool S16>
+BQ_DEV void gemm_epilogue(const GemmArgs &a, const void *sc, int e, int warp, int lane, uint32_t tmem,
                           uint32_t sbase, const GemmBars &B, volatile int *abort, int64_t row0, int tok0) {
   const int ngroups = (int)(a.K / G);
   const uint32_t d_full = B.d_full;
@@ -422,12 +430,12 @@ BQ_DEV void gemm_epilogue(const GemmArgs &a, const float *sc, int e, int warp, i
 #pragma unroll
   for (int i = 0; i < 64; ++i) acc[i] = 0.0f;
   const uint32_t lane_addr = ((uint32_t)(quad * 32) << 16);
-  float s_next = __ldg(sc + rloc);            // scale of group 0 (block-major metadata)
+  float s_next = load_scale<S16>(sc, rloc);   // scale of group 0 (block-major metadata)
   bool ok = true;
   for (int g = 0; g < ngroups; ++g) {
     const int buf = g & 1;
     const float s = s_next;
-    if (g + 1 < ngroups) s_next = __ldg(sc + (int64_t)(g + 1) * 128 + rloc);
+    if (g + 1 < ngroups) s_next = load_scale<S16>(sc, (int64_t)(g + 1) * 128 + rloc);
     // tcgen05.ld below is warp-collective: the whole warp leaves together
     if (!__all_sync(0xffffffffu, mbar_wait(d_full + 8u * buf, (g >> 1) & 1))) {
       *abort = 1;
@@ -464,8 +472,8 @@ BQ_DEV void gemm_epilogue(const GemmArgs &a, const float *sc, int e, int warp, i
 }
 
 // The roles of one CTA for a block of width BITS, group G.
-template <int XT, int BITS, int G>
-BQ_DEV void gemm_roles(const GemmArgs &a, const CUtensorMap *xmap, const uint8_t *pk, const float *sc,
+template <int XT, int BITS, int G, bool S16>
+BQ_DEV void gemm_roles(const GemmArgs &a, const CUtensorMap *xmap, const uint8_t *pk, const void *sc,
                        const uint8_t *ze, int warp, int lane, uint32_t tmem, uint32_t sbase, const GemmBars &B,
                        volatile int *abort, int64_t row0, int tok0) {
   if (warp < kGemmWarpDeq0) {
@@ -478,7 +486,7 @@ BQ_DEV void gemm_roles(const GemmArgs &a, const CUtensorMap *xmap, const uint8_t
     gemm_dequant<XT, BITS, G>(a, warp - kGemmWarpDeq0, lane, sbase, B, abort);
   } else {
     setmaxnreg_inc<kGemmRegsEpi>();
-    gemm_epilogue<XT, BITS, G>(a, sc, warp - kGemmWarpEpi0, warp, lane, tmem, sbase, B, abort, row0, tok0);
+    gemm_epilogue<XT, BITS, G, S16>(a, sc, warp - kGemmWarpEpi0, warp, lane, tmem, sbase, B, abort, row0, tok0);
   }
 }
 
@@ -488,9 +496,10 @@ BQ_DEV void gemm_roles(const GemmArgs &a, const CUtensorMap *xmap, const uint8_t
 // bits (group 64); the CTA's block has one width, so it runs that width's
 // roles, its codes and metadata found by running sums over the map (a block
 // of b bits holds 16 K b code bytes and 128 K / group metadata entries).
-template <int XT, int BITS, int G, bool MIXED>
+template <int XT, int BITS, int G, bool MIXED, bool S16 = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap xmap, const GemmArgs a) {
+  constexpr int SB = S16 ? 2 : 4;  // bytes per scale
   extern __shared__ __align__(1024) unsigned char gsm_raw[];
   // 1024-byte aligned base for the swizzled tiles
   const uint32_t raw = smem_u32(gsm_raw);
@@ -506,11 +515,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap xmap, const GemmArgs a) {
   // width of this block and where its codes / metadata start
   int bits = BITS;
   const uint8_t *pk;
-  const float *sc;
+  const uint8_t *sc;
   const uint8_t *ze;
   if (!MIXED) {
     pk = a.packed + blk * kGemmRowTile * a.K * BITS / 8;
-    sc = a.scales + blk * kGemmRowTile * (a.K / G);
+    sc = reinterpret_cast<const uint8_t *>(a.scales) + blk * kGemmRowTile * (a.K / G) * SB;
     ze = a.zeros + blk * kGemmRowTile * (a.K / G);
   } else {
     // every warp sums the map over the blocks before this one (shuffles)
@@ -527,7 +536,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap xmap, const GemmArgs a) {
     }
     bits = a.bit_map[blk];
     pk = a.packed + sb * 16 * a.K;
-    sc = a.scales + sg * a.K;
+    sc = reinterpret_cast<const uint8_t *>(a.scales) + sg * a.K * SB;
     ze = a.zeros + sg * a.K;
     if (bits != 4 && bits != 2) {  // the whole CTA leaves before allocating anything
       if (threadIdx.x == 0) bq_flag(BQ_FLAG_BADMAP);
@@ -566,8 +575,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap xmap, const GemmArgs a) {
   const uint32_t tmem = *tmem_slot;
 
   pdl_wait();
-  if (!MIXED || bits == BITS) gemm_roles<XT, BITS, G>(a, &xmap, pk, sc, ze, warp, lane, tmem, sbase, B, abort, row0, tok0);
-  else gemm_roles<XT, 2, 64>(a, &xmap, pk, sc, ze, warp, lane, tmem, sbase, B, abort, row0, tok0);
+  if (!MIXED || bits == BITS) gemm_roles<XT, BITS, G, S16>(a, &xmap, pk, sc, ze, warp, lane, tmem, sbase, B, abort, row0, tok0);
+  else gemm_roles<XT, 2, 64, S16>(a, &xmap, pk, sc, ze, warp, lane, tmem, sbase, B, abort, row0, tok0);
 
   // everything issued by this CTA has finished before the tensor memory goes
   tc_fence_before();

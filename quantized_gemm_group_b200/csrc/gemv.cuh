@@ -124,7 +124,8 @@ template <int BITS, int G> struct StageG {
 // Shared-memory layout (bytes), all staged per CTA:
 //   x     [M][KC + 8] 16-bit rows (only the real tokens), then a 16-byte
 //         zero chunk that ldmatrix reads for padding tokens
-//   meta  scales [KC/G][rows] fp32 then zeros [KC/G][rows] u8 of the block
+//   meta  scales [KC/G][rows] fp32 (or binary16) then zeros [KC/G][rows] u8
+//         of the block
 //   ring  `stages` x 16 KB of packed codes
 //   part  split-K receive buffer: S_k slices of ceil(TOK * rows / S_k) fp32
 //   bars  full[stages], empty[stages], x/meta barrier, abort flag
@@ -147,7 +148,7 @@ inline GemvSmem gemv_smem_layout(int M, int TOK, int64_t KC, int groups, int sta
 struct GemvArgs {
   const uint16_t *x;
   const uint8_t *packed;
-  const float *scales;
+  const void *scales;  // fp32, or binary16 when the kernel's S16 is set
   const uint8_t *zeros;
   const uint8_t *bit_map;
   uint16_t *y;
@@ -163,9 +164,10 @@ struct GemvArgs {
 // after lane 0 armed the stage's full barrier; stages the block's scales and
 // zeros for the slice (two copies, contiguous in the interleaved metadata
 // layout) and its x rows (one copy per token) once, on the x/meta barrier.
-// `pk`, `sc`, `ze` point at the block's first byte / element; `R` = row tiles.
-template <int BITS, int G>
-BQ_DEV void gemv_produce(const GemvArgs &a, const uint8_t *pk, const float *sc, const uint8_t *ze, int R,
+// `pk`, `sc`, `ze` point at the block's first byte (codes, scales of
+// SB bytes each, zeros); `R` = row tiles.
+template <int BITS, int G, int SB>
+BQ_DEV void gemv_produce(const GemvArgs &a, const uint8_t *pk, const uint8_t *sc, const uint8_t *ze, int R,
                          int64_t kc0, uint32_t smem, uint32_t bars, volatile int *abort, int lane) {
   using SG = StageG<BITS, G>;
   const int n = (int)(a.KC / SG::SC);
@@ -181,8 +183,8 @@ BQ_DEV void gemv_produce(const GemvArgs &a, const uint8_t *pk, const float *sc, 
   };
   auto stage_meta = [&]() {  // arms the x/meta barrier for metadata and x
     if (lane == 0) {
-      mbar_arrive_expect_tx(xm_full, (uint32_t)(groups * rows * 5 + a.M * a.KC * 2));
-      bulk_g2s(smem + a.L.s_off, sc + (kc0 / G) * rows, (uint32_t)(groups * rows * 4), xm_full);
+      mbar_arrive_expect_tx(xm_full, (uint32_t)(groups * rows * (SB + 1) + a.M * a.KC * 2));
+      bulk_g2s(smem + a.L.s_off, sc + (kc0 / G) * rows * SB, (uint32_t)(groups * rows * SB), xm_full);
       bulk_g2s(smem + a.L.z_off, ze + (kc0 / G) * rows, (uint32_t)(groups * rows), xm_full);
     }
     __syncwarp();
@@ -234,7 +236,7 @@ BQ_DEV void gemv_produce(const GemvArgs &a, const uint8_t *pk, const float *sc, 
 }
 
 // Consumer warp j: 16-row tile j of the CTA's block over the whole K-slice.
-template <int XT, int BITS, int G, int NB>
+template <int XT, int BITS, int G, int NB, int SB>
 BQ_DEV void gemv_consume(const GemvArgs &a, int j, int R, uint32_t smem, uint32_t bars, volatile int *abort,
                          int lane, float (&acc)[NB][4]) {
   using MT = MmaT<XT>;
@@ -266,7 +268,7 @@ BQ_DEV void gemv_consume(const GemvArgs &a, int j, int R, uint32_t smem, uint32_
     }
     return;
   }
-  const uint32_t stile = smem + a.L.s_off + (j * 16 + r) * 4;
+  const uint32_t stile = smem + a.L.s_off + (j * 16 + r) * SB;
   const uint32_t ztile = smem + a.L.z_off + j * 16 + r;
   int slot = 0, phase = 0;
   for (int i = 0; i < n; ++i) {
@@ -295,8 +297,16 @@ BQ_DEV void gemv_consume(const GemvArgs &a, int j, int R, uint32_t smem, uint32_
       const int g = i * SG::GPS + gi;  // group within the CTA's slice
       float s0, s1;
       uint32_t z0, z1;
-      asm volatile("ld.shared.f32 %0, [%1];" : "=f"(s0) : "r"(stile + g * rows * 4));
-      asm volatile("ld.shared.f32 %0, [%1];" : "=f"(s1) : "r"(stile + (g * rows + 8) * 4));
+      if (SB == 4) {
+        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(s0) : "r"(stile + g * rows * 4));
+        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(s1) : "r"(stile + (g * rows + 8) * 4));
+      } else {  // binary16 scales, exact in fp32
+        unsigned short h0, h1;
+        asm volatile("ld.shared.u16 %0, [%1];" : "=h"(h0) : "r"(stile + g * rows * 2));
+        asm volatile("ld.shared.u16 %0, [%1];" : "=h"(h1) : "r"(stile + (g * rows + 8) * 2));
+        s0 = __half2float(__ushort_as_half(h0));
+        s1 = __half2float(__ushort_as_half(h1));
+      }
       asm volatile("ld.shared.u8 %0, [%1];" : "=r"(z0) : "r"(ztile + g * rows));
       asm volatile("ld.shared.u8 %0, [%1];" : "=r"(z1) : "r"(ztile + g * rows + 8));
       // bf16 with at most 8 tokens: the operands are the exact integers
@@ -365,9 +375,10 @@ BQ_DEV void gemv_consume(const GemvArgs &a, int j, int R, uint32_t smem, uint32_
 // warps (8 consumers, one per 16-row tile of the block; warp 8 produces).
 // bit_map == nullptr: uniform BITS / G.  Otherwise one width per 128-row
 // block and the CTA runs (4, 128) or (2, 64).
-template <int XT, int BITS, int G, int NB, bool MIXED>
+template <int XT, int BITS, int G, int NB, bool MIXED, bool S16 = false>
 __global__ void __launch_bounds__(32 * (kGemvMaxConsumers + 1), 2)
 gemv_kernel(const GemvArgs a) {
+  constexpr int SB = S16 ? 2 : 4;  // bytes per scale
   using MT = MmaT<XT>;
   constexpr int TOK = 8 * NB;
   extern __shared__ __align__(128) unsigned char smem_raw[];
@@ -407,11 +418,11 @@ gemv_kernel(const GemvArgs a) {
   // width of this block and where its codes / metadata start
   int bits = BITS;
   const uint8_t *pk;
-  const float *sc;
+  const uint8_t *sc;
   const uint8_t *ze;
   if (!MIXED) {
     pk = a.packed + blk * 128 * a.K * BITS / 8;
-    sc = a.scales + blk * 128 * (a.K / G);
+    sc = reinterpret_cast<const uint8_t *>(a.scales) + blk * 128 * (a.K / G) * SB;
     ze = a.zeros + blk * 128 * (a.K / G);
   } else {
     int64_t sb = 0, sg = 0;
@@ -426,7 +437,7 @@ gemv_kernel(const GemvArgs a) {
       sg += __shfl_xor_sync(0xffffffffu, sg, off);
     }
     pk = a.packed + sb * 16 * a.K;
-    sc = a.scales + sg * a.K;
+    sc = reinterpret_cast<const uint8_t *>(a.scales) + sg * a.K * SB;
     ze = a.zeros + sg * a.K;
     bits = a.bit_map[blk];
     if (bits != 4 && bits != 2) {
@@ -443,14 +454,14 @@ gemv_kernel(const GemvArgs a) {
 
   if (warp == NC) {
     if (bits != 0) {
-      if (!MIXED) gemv_produce<BITS, G>(a, pk, sc, ze, R, kc0, smem, bars, abort, lane);
-      else if (bits == 4) gemv_produce<4, 128>(a, pk, sc, ze, R, kc0, smem, bars, abort, lane);
-      else gemv_produce<2, 64>(a, pk, sc, ze, R, kc0, smem, bars, abort, lane);
+      if (!MIXED) gemv_produce<BITS, G, SB>(a, pk, sc, ze, R, kc0, smem, bars, abort, lane);
+      else if (bits == 4) gemv_produce<4, 128, SB>(a, pk, sc, ze, R, kc0, smem, bars, abort, lane);
+      else gemv_produce<2, 64, SB>(a, pk, sc, ze, R, kc0, smem, bars, abort, lane);
     }
   } else if (bits != 0 && warp < R) {
-    if (!MIXED) gemv_consume<XT, BITS, G, NB>(a, warp, R, smem, bars, abort, lane, acc);
-    else if (bits == 4) gemv_consume<XT, 4, 128, NB>(a, warp, R, smem, bars, abort, lane, acc);
-    else gemv_consume<XT, 2, 64, NB>(a, warp, R, smem, bars, abort, lane, acc);
+    if (!MIXED) gemv_consume<XT, BITS, G, NB, SB>(a, warp, R, smem, bars, abort, lane, acc);
+    else if (bits == 4) gemv_consume<XT, 4, 128, NB, SB>(a, warp, R, smem, bars, abort, lane, acc);
+    else gemv_consume<XT, 2, 64, NB, SB>(a, warp, R, smem, bars, abort, lane, acc);
   }
 
   if (SK == 1) {

@@ -67,7 +67,7 @@ BQ_DEV uint32_t quant8_canonical(uint4 v, bool active, float *s_out, uint8_t *z_
 template <int WT, int BITS, int G, int UNROLL, int SCHEME = 0>
 __global__ void __launch_bounds__(256)
 quantize_canonical_kernel(const uint16_t *__restrict__ W, int64_t elems,
-                          uint8_t *__restrict__ packed, float *__restrict__ scales,
+                          uint8_t *__restrict__ packed, void *__restrict__ scales,
                           uint8_t *__restrict__ zeros) {
   constexpr int LANES = G / 8;
   const int lane = threadIdx.x & 31;
@@ -99,7 +99,7 @@ quantize_canonical_kernel(const uint16_t *__restrict__ W, int64_t elems,
         reinterpret_cast<uint16_t *>(packed)[e / 8] = (uint16_t)pk;
       }
       if ((lane % LANES) == 0) {
-        scales[e / G] = s;
+        store_scale<SCHEME>(scales, e / G, s);
         zeros[e / G] = z;
       }
     }
@@ -205,7 +205,7 @@ BQ_DEV void codes_of_group(const UnitRegs<BITS, G> &u, int h, int gi, const Grou
 // parameters from the lane that computed them by shuffle.
 template <int WT, int BITS, int G, int SCHEME = 0>
 BQ_DEV bool quantize_unit(const UnitRegs<BITS, G> &u, int64_t N, int64_t K, int64_t row0, int64_t col0,
-                          uint8_t *__restrict__ packed, float *__restrict__ scales,
+                          uint8_t *__restrict__ packed, void *__restrict__ scales,
                           uint8_t *__restrict__ zeros, int lane) {
   using UG = UnitGeom<BITS, G>;
   using E = Elem<WT>;
@@ -272,7 +272,7 @@ BQ_DEV bool quantize_unit(const UnitRegs<BITS, G> &u, int64_t N, int64_t K, int6
     if (HALF >= 2 || !up1) {  // with C = 2, lanes c and c ^ 1 hold the same combination
       const int k = base + i, h = k / NG, gi = k % NG;
       const int64_t idx = il_meta_index(row0 + r + 8 * h, col0 / G + gi, N, GK);
-      scales[idx] = own[i].s;
+      store_scale<SCHEME>(scales, idx, own[i].s);
       zeros[idx] = (uint8_t)own[i].z;
     }
   }
@@ -347,7 +347,7 @@ BQ_DEV void load_unit_smem(UnitRegs<BITS, G> &u, uint32_t su, int t, int lane) {
 template <int WT, int BITS, int G, int SCHEME = 0>
 __global__ void __launch_bounds__(kQtThreads, qt_ctas_per_sm<G>())
 quantize_tma_kernel(const __grid_constant__ CUtensorMap wmap, int64_t N, int64_t K, int stages,
-                    uint8_t *__restrict__ packed, float *__restrict__ scales, uint8_t *__restrict__ zeros) {
+                    uint8_t *__restrict__ packed, void *__restrict__ scales, uint8_t *__restrict__ zeros) {
   using UG = UnitGeom<BITS, G>;
   constexpr uint32_t SU_BYTES = (uint32_t)(UG::U / 64) * 8192u;
   extern __shared__ __align__(1024) unsigned char qt_raw[];
