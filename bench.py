@@ -65,13 +65,14 @@ METRIC = "W4/W2 dequant-GEMV weight GB/s (M<=16) & GEMM TFLOP/s (M>=2048) vs roo
 # helpers
 # ---------------------------------------------------------------------------
 
-def weight_bytes(N, K, bits, group):
-    """Algorithmic bytes of one decode linear's weights: codes + fp32 scale + u8 zero."""
-    return N * K * bits // 8 + N * (K // group) * 5
+def weight_bytes(N, K, bits, group, scale_bytes=4):
+    """Algorithmic bytes of one decode linear's weights: codes + scale (fp32, or
+    binary16) + u8 zero per group."""
+    return N * K * bits // 8 + N * (K // group) * (scale_bytes + 1)
 
 
-def linear_bytes(N, K, bits, group, M):
-    return weight_bytes(N, K, bits, group) + 2 * M * K + 2 * M * N
+def linear_bytes(N, K, bits, group, M, scale_bytes=4):
+    return weight_bytes(N, K, bits, group, scale_bytes) + 2 * M * K + 2 * M * N
 
 
 def peaks():
@@ -194,8 +195,10 @@ def fused_shapes(layers):
 class Stack:
     """The quantized decode stack resident in HBM, plus per-M activations."""
 
-    def __init__(self, layers, bits, group, seed_offset, dist_kind, quant_time=True):
+    def __init__(self, layers, bits, group, seed_offset, dist_kind, quant_time=True, scheme="asymmetric"):
         self.layers, self.bits, self.group = layers, bits, group
+        self.scheme = scheme
+        self.scale_bytes = 2 if scheme == "asymmetric_f16_scale" else 4
         self.shapes = stack_shapes(layers)
         dev = "cuda"
         # fp16 weights for the whole stack (~14 GB at 32 layers) so the
@@ -216,7 +219,8 @@ class Stack:
         nlin = len(synth.LLAMA3_8B_LINEARS)
         for (l, fname, N, K, mods) in self.fused:
             pk = torch.empty(bq.bq_packed_bytes(N, K, bits), dtype=torch.uint8, device=dev)
-            sc = torch.empty(N * (K // group), dtype=torch.float32, device=dev)
+            sc = torch.empty(N * (K // group), dtype=torch.float16 if self.scale_bytes == 2 else torch.float32,
+                             device=dev)
             ze = torch.empty(N * (K // group), dtype=torch.uint8, device=dev)
             self.fq.append((pk, sc, ze))
             r0 = 0
@@ -227,7 +231,7 @@ class Stack:
                 self.q[l * nlin + m] = (pk[cb:ce], sc[gb:ge], ze[gb:ge])
                 r0 += Nm
         for W, (l, mi, name, N, K), out in zip(Ws, self.shapes, self.q):
-            bq.bq_quantize(W, bits, group, "interleaved", out=out)
+            bq.bq_quantize(W, bits, group, "interleaved", out=out, scheme=scheme)
         torch.cuda.synchronize()
         if bq.bq_device_status() != bq.BQ_OK:
             raise RuntimeError("quantizer reported a device error")
@@ -244,11 +248,11 @@ class Stack:
         s.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(s):
             for W, out in zip(Ws, self.q):            # warm
-                bq.bq_quantize(W, self.bits, self.group, "interleaved", out=out, stream=s)
+                bq.bq_quantize(W, self.bits, self.group, "interleaved", out=out, stream=s, scheme=self.scheme)
             s.synchronize()
             with torch.cuda.graph(g, stream=s):
                 for W, out in zip(Ws, self.q):
-                    bq.bq_quantize(W, self.bits, self.group, "interleaved", out=out, stream=s)
+                    bq.bq_quantize(W, self.bits, self.group, "interleaved", out=out, stream=s, scheme=self.scheme)
         torch.cuda.current_stream().wait_stream(s)
         g.replay()
         torch.cuda.synchronize()
@@ -262,7 +266,8 @@ class Stack:
             times.append(a.elapsed_time(b) / 1e3)
         t = min(times)
         weights = sum(N * K for (_, _, _, N, K) in self.shapes)
-        byts = sum(N * K * 2 + weight_bytes(N, K, self.bits, self.group) for (_, _, _, N, K) in self.shapes)
+        byts = sum(N * K * 2 + weight_bytes(N, K, self.bits, self.group, self.scale_bytes)
+                   for (_, _, _, N, K) in self.shapes)
         del g
         return {"weights": weights, "seconds": t, "weights_per_s": weights / t, "GBps": byts / t / 1e9,
                 "bytes": byts, "launches": len(self.shapes)}
@@ -283,7 +288,8 @@ class Stack:
         return g
 
     def step_bytes(self, Ms):
-        return sum(linear_bytes(N, K, self.bits, self.group, M) for M in Ms for (_, _, N, K, _) in self.fused)
+        return sum(linear_bytes(N, K, self.bits, self.group, M, self.scale_bytes)
+                   for M in Ms for (_, _, N, K, _) in self.fused)
 
 
 def time_graph(g, steps, warmup, stream, world, profile=False):
@@ -565,6 +571,12 @@ def quant_shape_numbers(hbm, reps=10):
     res[f"quantize_symmetric {N}x{K} INT4 g128"] = {"us": round(t * 1e6, 1), "GBps": round(byts / t / 1e9, 1),
                                                    "frac_of_measured_hbm": round(byts / t / 1e9 / hbm, 4)}
     del out
+    out = bq.bq_quantize(W, 2, 64, "interleaved", scheme="asymmetric_f16_scale")
+    t = timed(lambda: bq.bq_quantize(W, 2, 64, "interleaved", out=out, scheme="asymmetric_f16_scale"))
+    byts = N * K * 2 + weight_bytes(N, K, 2, 64, scale_bytes=2)
+    res[f"quantize_f16_scales {N}x{K} INT2 g64"] = {"us": round(t * 1e6, 1), "GBps": round(byts / t / 1e9, 1),
+                                                   "frac_of_measured_hbm": round(byts / t / 1e9 / hbm, 4)}
+    del out
     fq = torch.empty_like(W)
     t = timed(lambda: bq.bq_fake_quantize(W, 4, 128, out=fq))
     byts = N * K * 4
@@ -792,6 +804,18 @@ def run_gpu(args, world, rank, local):
             "quantizer_stack": quant_summary(other.quant) if other.quant else None}
         del other
         torch.cuda.empty_cache()
+    if not args.no_f16_scale:
+        # the INT2 g64 stack again with binary16 group scales (3 instead of 5
+        # metadata bytes per group): quantizer and decode numbers
+        f16s = Stack(args.layers, 2, 64, seed_offset=rank * 100000 + 7, dist_kind="t4",
+                     quant_time=not args.no_quant, scheme="asymmetric_f16_scale")
+        extra["int2_stack_f16_scales"] = {
+            "weights": "fp16 Student-t4 std 0.02 + 0.1% x10 outlier cols", "group": 64,
+            "bytes_per_weight": round(0.25 + 3 / 64, 5),
+            "per_M": stack_per_m(f16s, Ms, hbm, max(2, args.steps), world),
+            "quantizer_stack": quant_summary(f16s.quant) if f16s.quant else None}
+        del f16s
+        torch.cuda.empty_cache()
     if not args.no_mixed:
         extra["mixed_stack"] = mixed_numbers(args.layers, (1, 16), hbm)
     if args.split:
@@ -979,6 +1003,7 @@ def main():
     ap.add_argument("--no-gemm", action="store_true", help="skip the prefill GEMM numbers")
     ap.add_argument("--no-grad", action="store_true", help="skip the input-gradient (backward) numbers")
     ap.add_argument("--no-mixed", action="store_true", help="skip the Layer-mix / Channel-mix decode stacks")
+    ap.add_argument("--no-f16-scale", action="store_true", help="skip the INT2 stack with binary16 scales")
     ap.add_argument("--no-other-width", action="store_true",
                     help="skip the second stack at the other width (INT2 g64 when timing INT4)")
     ap.add_argument("--split", action="store_true",
