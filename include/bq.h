@@ -262,8 +262,11 @@ bq_status bq_linear_f16s(const void *x, bq_dtype xtype, int64_t M, int64_t K,
  *   dy       [M, N] of dtype (BQ_BF16 or BQ_F16), 16-byte aligned
  *   packed / scales / zeros: W from bq_quantize or bq_quantize_symmetric in
  *            BQ_LAYOUT_INTERLEAVED, all three 16-byte aligned
- *   bit_map  must be NULL (uniform width; BQ_ERR_UNSUPPORTED otherwise);
- *            bits / group as in bq_linear
+ *   bit_map  NULL for a uniform matrix (bits, group as in bq_linear), else a
+ *            DEVICE width map as in bq_quantize_mixed (W from
+ *            bq_quantize_mixed; bits, group ignored; N % 128 == 0; an entry
+ *            other than 4 or 2 sets BQ_ERR_UNSUPPORTED in the device status
+ *            and that block contributes nothing)
  *   dx       [M, K] of dtype, written in full (N == 0: zeros, dy not read;
  *            M == 0 or K == 0: nothing is done)
  * dx[m, k] = sum_n dy[m, n] s[n, g] (q[n, k] - z[n, g]) on tensor cores with

@@ -237,14 +237,14 @@ def bq_linear(x: torch.Tensor, packed, scales, zeros, N: int, bits: int = 4, gro
 
 
 def bq_linear_grad_input(dy: torch.Tensor, packed, scales, zeros, K: int, bits: int = 4, group: int | None = None,
-                         layout: str = "interleaved", out=None, stream=None):
+                         layout: str = "interleaved", out=None, stream=None, bit_map_dev=None):
     """dx [M, K] = dy [M, N] . dequant(W), dx in dy's dtype (the input
-    gradient of bq_linear)."""
+    gradient of bq_linear); bit_map_dev: a width map's device copy, as for bq_linear."""
     group = group or GROUP_OF_BITS.get(bits, 0)
     M, N = dy.shape
     dx = out if out is not None else torch.empty((M, K), dtype=dy.dtype, device=dy.device)
     st = lib().bq_linear_grad_input(_ptr(dy), DTYPE_CODE[dy.dtype], M, N, _ptr(packed), _ptr(scales), _ptr(zeros),
-                                    None, bits, group, K, LAYOUTS[layout], _ptr(dx), _stream(stream))
+                                    _ptr(bit_map_dev), bits, group, K, LAYOUTS[layout], _ptr(dx), _stream(stream))
     _check("bq_linear_grad_input", st)
     return dx
 

@@ -421,11 +421,12 @@ GradGeom grad_geometry(int M, int64_t N, int64_t K, int gmax) {
   return g;
 }
 
-template <int XT, int BITS, int G, int NB>
+template <int XT, int BITS, int G, int NB, bool MIXED = false>
 bq_status launch_grad_t(const GradGeom &g, GradArgs a, cudaStream_t st) {
-  auto kern = grad_input_kernel<XT, BITS, G, NB>;
-  if (!ensure_smem<grad_input_kernel<XT, BITS, G, NB>>(kMaxSmem)) return BQ_ERR_CUDA;
-  constexpr int gmax = (G <= kGradSlice) ? kGradSlice / G : 1;
+  auto kern = grad_input_kernel<XT, BITS, G, NB, MIXED>;
+  if (!ensure_smem<grad_input_kernel<XT, BITS, G, NB, MIXED>>(kMaxSmem)) return BQ_ERR_CUDA;
+  // metadata groups per 128-column slice: a width map's 2-bit blocks have two
+  constexpr int gmax = MIXED ? 2 : ((G <= kGradSlice) ? kGradSlice / G : 1);
   a.stages = g.stages;
   a.L = grad_smem_layout(a.M, 8 * NB, gmax, g.stages, g.d);
   if (a.L.total > kMaxSmem) return BQ_ERR_SHAPE;
@@ -460,16 +461,22 @@ bq_status launch_grad_t(const GradGeom &g, GradArgs a, cudaStream_t st) {
 
 template <int XT>
 bq_status grad_dispatch(const uint16_t *dy, int M, int64_t N, const uint8_t *packed, const float *scales,
-                        const uint8_t *zeros, int bits, int group, int64_t K, uint16_t *dx, cudaStream_t st) {
+                        const uint8_t *zeros, const uint8_t *bit_map, int bits, int group, int64_t K, uint16_t *dx,
+                        cudaStream_t st) {
   GradArgs a = {};
   a.dy = dy;
   a.packed = packed;
   a.scales = scales;
   a.zeros = zeros;
+  a.bit_map = bit_map;
   a.dx = dx;
   a.N = N;
   a.K = K;
   a.M = M;
+  if (bit_map) {  // width map: the 4-bit kernel with per-block widths
+    const GradGeom g = grad_geometry(M, N, K, 2);
+    return g.NB == 1 ? launch_grad_t<XT, 4, 128, 1, true>(g, a, st) : launch_grad_t<XT, 4, 128, 2, true>(g, a, st);
+  }
 #define BQ_GD(B, G_)                                                                  \
   if (bits == B && group == G_) {                                                     \
     const GradGeom g = grad_geometry(M, N, K, (G_ <= kGradSlice) ? kGradSlice / G_ : 1); \
@@ -824,9 +831,13 @@ bq_status bq_linear_grad_input(const void *dy, bq_dtype dtype, int64_t M, int64_
                                int group, int64_t K, bq_layout layout, void *dx, void *stream) {
   if (M < 0 || K < 0 || N < 0) return BQ_ERR_SHAPE;
   if (dtype != BQ_F16 && dtype != BQ_BF16) return BQ_ERR_UNSUPPORTED;
-  if (layout != BQ_LAYOUT_INTERLEAVED || bit_map) return BQ_ERR_UNSUPPORTED;
-  if (!valid_bits(bits) || !linear_group_ok(bits, group)) return BQ_ERR_UNSUPPORTED;
-  if (N % 16 || K % kGradSlice || K % group) return BQ_ERR_SHAPE;
+  if (layout != BQ_LAYOUT_INTERLEAVED) return BQ_ERR_UNSUPPORTED;
+  if (bit_map) {
+    if (N % 128 || K % kGradSlice) return BQ_ERR_SHAPE;
+  } else {
+    if (!valid_bits(bits) || !linear_group_ok(bits, group)) return BQ_ERR_UNSUPPORTED;
+    if (N % 16 || K % kGradSlice || K % group) return BQ_ERR_SHAPE;
+  }
   if (M == 0 || K == 0) return BQ_OK;
   if (!dx) return BQ_ERR_NULL;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -842,8 +853,9 @@ bq_status bq_linear_grad_input(const void *dy, bq_dtype dtype, int64_t M, int64_
   for (int64_t m0 = 0; m0 < M; m0 += 16) {
     const int mb = (int)((M - m0) < 16 ? (M - m0) : 16);
     bq_status s = (dtype == BQ_BF16)
-                      ? grad_dispatch<1>(g + m0 * N, mb, N, pk, scales, zeros, bits, group, K, out + m0 * K, st)
-                      : grad_dispatch<0>(g + m0 * N, mb, N, pk, scales, zeros, bits, group, K, out + m0 * K, st);
+                      ? grad_dispatch<1>(g + m0 * N, mb, N, pk, scales, zeros, bit_map, bits, group, K, out + m0 * K, st)
+                      : grad_dispatch<0>(g + m0 * N, mb, N, pk, scales, zeros, bit_map, bits, group, K, out + m0 * K,
+                                         st);
     if (s != BQ_OK) return s;
   }
   return BQ_OK;

@@ -87,6 +87,7 @@ struct GradArgs {
   const uint8_t *packed;
   const float *scales;
   const uint8_t *zeros;
+  const uint8_t *bit_map;  // width map (one entry per 128-row block), or null
   uint16_t *dx;
   int64_t N, K;
   int M;
@@ -124,28 +125,56 @@ template <int XT> BQ_DEV float elem16_to_f32(uint32_t h);
 template <> BQ_DEV float elem16_to_f32<1>(uint32_t h) { return __uint_as_float(h << 16); }
 template <> BQ_DEV float elem16_to_f32<0>(uint32_t h) { return __half2float(__ushort_as_half((unsigned short)h)); }
 
-// Producer warp: blocks [b0, b0 + nblk) of the CTA's column slice.
-template <int BITS, int G>
+// Producer warp: blocks [b0, b0 + nblk) of the CTA's column slice.  Under a
+// width map (MIXED) each block has its own width (4 bits / group 128 or 2
+// bits / group 64); its codes and metadata start after the blocks before it:
+// a block of b bits holds 16 K b code bytes and 128 K / group metadata
+// entries (running sums, from a warp reduction over the map up to b0).
+template <int BITS, int G, bool MIXED>
 BQ_DEV void grad_produce(const GradArgs &a, int64_t b0, int nblk, int64_t col0, uint32_t smem, uint32_t bars,
                          volatile int *abort, int lane) {
-  constexpr int T = (BITS == 4) ? 64 : 128;
-  constexpr int TPS = kGradSlice / T;                            // column tiles in the slice
-  constexpr int GPS = (G <= kGradSlice) ? kGradSlice / G : 1;    // groups in the slice
   const int S = a.stages;
-  const int64_t Gt = a.K / G;
-  const int64_t gs = col0 / G;
+  int64_t sb = 0, sg = 0;  // bits and group units (1 per 4-bit, 2 per 2-bit block) before block b0 + i
+  if (MIXED) {
+    for (int64_t jb = lane; jb < b0; jb += 32) {
+      const int b = a.bit_map[jb];
+      sb += b;
+      sg += (b == 4) ? 1 : 2;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      sb += __shfl_xor_sync(0xffffffffu, sb, off);
+      sg += __shfl_xor_sync(0xffffffffu, sg, off);
+    }
+  }
   auto stage_of = [&](int i) { return smem + (uint32_t)((i % S) * a.L.sb); };
-  auto issue_weights = [&](int i) {  // lane 0: arm the stage, copy codes and metadata
+  auto issue_weights = [&](int i) {  // lane 0, blocks in order: arm the stage, copy codes and metadata
     const int64_t blk = b0 + i;
     const int rows = grad_block_rows(a.N, blk);
     const int R = rows / 16;
     const uint32_t st = stage_of(i), full = bars + 8u * (i % S);
+    const int bits = MIXED ? a.bit_map[blk] : BITS;
+    if (MIXED && bits != 4 && bits != 2) {  // not a width: flag it, the stage carries dy only
+      bq_flag(BQ_FLAG_BADMAP);
+      mbar_arrive_expect_tx(full, (uint32_t)(a.M * rows * 2));
+      sb += bits;
+      sg += 2;
+      return;
+    }
+    const int g = MIXED ? (bits == 4 ? 128 : 64) : G;
+    const int T = (bits == 4) ? 64 : 128;
+    const int TPS = kGradSlice / T;                                // column tiles in the slice
+    const int GPS = (g <= kGradSlice) ? kGradSlice / g : 1;        // groups in the slice
     const uint32_t cb = (uint32_t)(TPS * R * 512);
     mbar_arrive_expect_tx(full, cb + (uint32_t)(GPS * rows * 5 + a.M * rows * 2));
-    bulk_g2s(st, a.packed + blk * 128 * a.K * BITS / 8 + (col0 / T) * R * 512, cb, full);
-    const int64_t mi = 128 * Gt * blk + gs * rows;
+    const int64_t code0 = MIXED ? 16 * a.K * sb : blk * 128 * a.K * BITS / 8;
+    const int64_t meta0 = MIXED ? a.K * sg : 128 * (a.K / G) * blk;
+    bulk_g2s(st, a.packed + code0 + (col0 / T) * R * 512, cb, full);
+    const int64_t mi = meta0 + (col0 / g) * rows;
     bulk_g2s(st + a.L.s_off, a.scales + mi, (uint32_t)(GPS * rows * 4), full);
     bulk_g2s(st + a.L.z_off, a.zeros + mi, (uint32_t)(GPS * rows), full);
+    sb += bits;
+    sg += (bits == 4) ? 1 : 2;
   };
   auto issue_dy = [&](int i) {  // one dy row per lane
     const int64_t blk = b0 + i;
@@ -190,10 +219,14 @@ BQ_DEV void grad_produce(const GradArgs &a, int64_t b0, int nblk, int64_t col0, 
 // sums (16 tokens x 64 columns) stay in registers.  acc[run][token block]
 // [fragment] accumulates dx^T for the warp's runs: fragment q is column
 // 16 run + 2 (g % 4) + 8 (g / 4) + q / 2 and token 8 nb + 2t + (q % 2), times
-// 2^(2 BITS (g / 4)) (undone when the sums leave the registers).
-template <int XT, int BITS, int G, int NB, int CW>
-BQ_DEV void grad_consume(const GradArgs &a, int w, int64_t b0, int nblk, uint32_t smem, uint32_t bars,
-                         volatile int *abort, int lane, float (&acc)[8 / CW][NB][4]) {
+// 2^(2 ACC_BITS (g / 4)) (undone when the sums leave the registers).  A block
+// of BITS < ACC_BITS (a width map's 2-bit blocks) has its codes at 2 BITS (g / 4)
+// and makes up the difference on its A operand, whose rows g and g + 8 are the
+// lane's columns (an exact power of two on an exact small integer).
+// One staged block `st` of `rows` rows.
+template <int XT, int BITS, int G, int NB, int CW, int ACC_BITS>
+BQ_DEV void grad_consume_block(const GradArgs &a, int w, uint32_t st, int rows, int lane,
+                               float (&acc)[8 / CW][NB][4]) {
   constexpr int T = (BITS == 4) ? 64 : 128;
   constexpr int RPT = T / 16;                                     // runs per column tile
   constexpr int RPG = ((G <= kGradSlice) ? G : kGradSlice) / 16;  // runs per group in the slice
@@ -203,7 +236,6 @@ BQ_DEV void grad_consume(const GradArgs &a, int w, int64_t b0, int nblk, uint32_
   constexpr uint32_t QM = (1u << BITS) - 1;
   constexpr uint32_t kMagic = 0x4B000000u;                        // fp32 2^23
   const int g = lane >> 2, t = lane & 3;
-  const int S = a.stages;
   const int r_lo = (w % CW) * RW;                                 // the warp's first run
   const int rt0 = (w / CW) * CW;                                  // the warp's first row tile
   // lane group g takes the column pair (2 (g % 4) + 8 (g / 4), + 1) of every
@@ -213,6 +245,84 @@ BQ_DEV void grad_consume(const GradArgs &a, int w, int64_t b0, int nblk, uint32_
   const uint32_t slot1 = 16u * (uint32_t)(4 * t + (g & 3));       // rows t, t + 8
   const uint32_t slot2 = slot1 + 16u * 16u;                       // rows t + 4, t + 12
   const uint32_t hpos = 2u * BITS * (uint32_t)(g >> 2);
+  // 2^(2 (ACC_BITS - BITS) (g / 4)): the accumulators' convention for this lane's columns
+  const float acc_fix = (ACC_BITS != BITS && (g >> 2)) ? (float)(1 << (2 * (ACC_BITS - BITS))) : 1.0f;
+  const int R = rows / 16;
+#pragma unroll
+  for (int rti = 0; rti < CW; ++rti) {
+    const int rt = rt0 + rti;
+    if (rt >= R) break;
+#pragma unroll
+    for (int j = 0; j < GW; ++j) {
+      const int gi = r_lo / RPG + j;  // group within the slice
+      // the lane's rows in this tile: 16 rt + t + 4 aa + 8 h
+      uint32_t bp[NB][2][2];
+      float cz[2][2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int aa = 0; aa < 2; ++aa) {
+          const int nl = 16 * rt + t + 4 * aa + 8 * h;
+          float s;
+          uint32_t z;
+          asm volatile("ld.shared.f32 %0, [%1];" : "=f"(s) : "r"(st + a.L.s_off + (gi * rows + nl) * 4));
+          asm volatile("ld.shared.u8 %0, [%1];" : "=r"(z) : "r"(st + a.L.z_off + gi * rows + nl));
+          // the second half tile's codes sit BITS bits higher: scale its dy' down by 2^BITS
+          const float sh = h ? s * (1.0f / (float)(1 << BITS)) : s;
+          cz[h][aa] = __uint_as_float(kMagic | (z << (BITS * h + hpos)));  // 2^23 + z 2^(BITS h + hpos)
+#pragma unroll
+          for (int nb = 0; nb < NB; ++nb) {
+            const int m = g + 8 * nb;
+            float dyv = 0.0f;
+            if (m < a.M) {
+              uint32_t hbits;
+              asm volatile("ld.shared.u16 %0, [%1];" : "=r"(hbits) : "r"(st + a.L.dy_off + m * kGradDyStride + nl * 2));
+              dyv = elem16_to_f32<XT>(hbits);
+            }
+            bp[nb][h][aa] = to_tf32(__fmul_rn(dyv, sh));
+          }
+        }
+#pragma unroll
+      for (int rr = 0; rr < RPGW; ++rr) {
+        const int rl = j * RPGW + rr;  // run within the warp's range
+        const int rs = r_lo + rl;      // run within the slice
+        const int ct = rs / RPT;       // column tile
+        const int wj = (BITS == 4) ? (rs % RPT) : (rs % RPT) / 2;
+        const uint32_t tb = st + (uint32_t)((ct * R + rt) * 512 + wj * 4);
+        uint32_t w1 = lds_u32(tb + slot1), w2 = lds_u32(tb + slot2);
+        // 2 bits: the word's second run sits 8 bits higher (r_lo is even, so
+        // the parity of rs is that of rl)
+        if (BITS == 2 && (rl & 1)) {
+          w1 >>= 8;
+          w2 >>= 8;
+        }
+        const uint32_t w1o = w1 >> 16, w2o = w2 >> 16;  // odd columns
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t mask = QM << (BITS * h + hpos);
+          uint32_t av[4];
+          av[0] = __float_as_uint(__fsub_rn(__uint_as_float(and_or(w1, mask, kMagic)), cz[h][0]));
+          av[1] = __float_as_uint(__fsub_rn(__uint_as_float(and_or(w1o, mask, kMagic)), cz[h][0]));
+          av[2] = __float_as_uint(__fsub_rn(__uint_as_float(and_or(w2, mask, kMagic)), cz[h][1]));
+          av[3] = __float_as_uint(__fsub_rn(__uint_as_float(and_or(w2o, mask, kMagic)), cz[h][1]));
+          if (ACC_BITS != BITS) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) av[q] = __float_as_uint(__uint_as_float(av[q]) * acc_fix);
+          }
+#pragma unroll
+          for (int nb = 0; nb < NB; ++nb) mma_tf32(acc[rl][nb], av, bp[nb][h][0], bp[nb][h][1]);
+        }
+      }
+    }
+  }
+}
+
+// The consumer loop: blocks [b0, b0 + nblk); under a width map (MIXED) each
+// block runs its own width's body, with the 4-bit accumulator convention.
+template <int XT, int BITS, int G, int NB, int CW, bool MIXED>
+BQ_DEV void grad_consume(const GradArgs &a, int w, int64_t b0, int nblk, uint32_t smem, uint32_t bars,
+                         volatile int *abort, int lane, float (&acc)[8 / CW][NB][4]) {
+  const int S = a.stages;
   for (int i = 0; i < nblk; ++i) {
     const uint32_t st = smem + (uint32_t)((i % S) * a.L.sb);
     const uint32_t full = bars + 8u * (i % S), empty = bars + 8u * (S + i % S);
@@ -225,69 +335,12 @@ BQ_DEV void grad_consume(const GradArgs &a, int w, int64_t b0, int nblk, uint32_
       break;
     }
     const int rows = grad_block_rows(a.N, b0 + i);
-    const int R = rows / 16;
-#pragma unroll
-    for (int rti = 0; rti < CW; ++rti) {
-      const int rt = rt0 + rti;
-      if (rt >= R) break;
-#pragma unroll
-      for (int j = 0; j < GW; ++j) {
-        const int gi = r_lo / RPG + j;  // group within the slice
-        // the lane's rows in this tile: 16 rt + t + 4 aa + 8 h
-        uint32_t bp[NB][2][2];
-        float cz[2][2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-          for (int aa = 0; aa < 2; ++aa) {
-            const int nl = 16 * rt + t + 4 * aa + 8 * h;
-            float s;
-            uint32_t z;
-            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(s) : "r"(st + a.L.s_off + (gi * rows + nl) * 4));
-            asm volatile("ld.shared.u8 %0, [%1];" : "=r"(z) : "r"(st + a.L.z_off + gi * rows + nl));
-            // the second half tile's codes sit BITS bits higher: scale its dy' down by 2^BITS
-            const float sh = h ? s * (1.0f / (float)(1 << BITS)) : s;
-            cz[h][aa] = __uint_as_float(kMagic | (z << (BITS * h + hpos)));  // 2^23 + z 2^(BITS h + hpos)
-#pragma unroll
-            for (int nb = 0; nb < NB; ++nb) {
-              const int m = g + 8 * nb;
-              float dyv = 0.0f;
-              if (m < a.M) {
-                uint32_t hbits;
-                asm volatile("ld.shared.u16 %0, [%1];" : "=r"(hbits) : "r"(st + a.L.dy_off + m * kGradDyStride + nl * 2));
-                dyv = elem16_to_f32<XT>(hbits);
-              }
-              bp[nb][h][aa] = to_tf32(__fmul_rn(dyv, sh));
-            }
-          }
-#pragma unroll
-        for (int rr = 0; rr < RPGW; ++rr) {
-          const int rl = j * RPGW + rr;  // run within the warp's range
-          const int rs = r_lo + rl;      // run within the slice
-          const int ct = rs / RPT;       // column tile
-          const int wj = (BITS == 4) ? (rs % RPT) : (rs % RPT) / 2;
-          const uint32_t tb = st + (uint32_t)((ct * R + rt) * 512 + wj * 4);
-          uint32_t w1 = lds_u32(tb + slot1), w2 = lds_u32(tb + slot2);
-          // 2 bits: the word's second run sits 8 bits higher (r_lo is even, so
-          // the parity of rs is that of rl)
-          if (BITS == 2 && (rl & 1)) {
-            w1 >>= 8;
-            w2 >>= 8;
-          }
-          const uint32_t w1o = w1 >> 16, w2o = w2 >> 16;  // odd columns
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint32_t mask = QM << (BITS * h + hpos);
-            uint32_t av[4];
-            av[0] = __float_as_uint(__fsub_rn(__uint_as_float(and_or(w1, mask, kMagic)), cz[h][0]));
-            av[1] = __float_as_uint(__fsub_rn(__uint_as_float(and_or(w1o, mask, kMagic)), cz[h][0]));
-            av[2] = __float_as_uint(__fsub_rn(__uint_as_float(and_or(w2, mask, kMagic)), cz[h][1]));
-            av[3] = __float_as_uint(__fsub_rn(__uint_as_float(and_or(w2o, mask, kMagic)), cz[h][1]));
-#pragma unroll
-            for (int nb = 0; nb < NB; ++nb) mma_tf32(acc[rl][nb], av, bp[nb][h][0], bp[nb][h][1]);
-          }
-        }
-      }
+    if (!MIXED) {
+      grad_consume_block<XT, BITS, G, NB, CW, BITS>(a, w, st, rows, lane, acc);
+    } else {
+      const int bits = a.bit_map[b0 + i];
+      if (bits == 4) grad_consume_block<XT, 4, 128, NB, CW, 4>(a, w, st, rows, lane, acc);
+      else if (bits == 2) grad_consume_block<XT, 2, 64, NB, CW, 4>(a, w, st, rows, lane, acc);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(empty);
@@ -297,7 +350,7 @@ BQ_DEV void grad_consume(const GradArgs &a, int w, int64_t b0, int nblk, uint32_
 // Kernel.  grid = (K / 128, d); cluster = (1, d, 1); block = 9 warps (8
 // consumers, warp 8 produces).  Cluster rank r streams the blocks
 // [r nb / d, (r + 1) nb / d) of the nb = ceil(N / 128) row blocks.
-template <int XT, int BITS, int G, int NB>
+template <int XT, int BITS, int G, int NB, bool MIXED = false>
 __global__ void __launch_bounds__(32 * (kGradWarps + 1), 2) grad_input_kernel(const GradArgs a) {
   using MT = MmaT<XT>;
   constexpr int TOK = 8 * NB;
@@ -339,8 +392,8 @@ __global__ void __launch_bounds__(32 * (kGradWarps + 1), 2) grad_input_kernel(co
 #pragma unroll
       for (int q = 0; q < 4; ++q) acc[r][nb][q] = 0.0f;
 
-  if (warp == kGradWarps) grad_produce<BITS, G>(a, b0, nblk, col0, smem, bars, abort, lane);
-  else grad_consume<XT, BITS, G, NB, CW>(a, warp, b0, nblk, smem, bars, abort, lane, acc);
+  if (warp == kGradWarps) grad_produce<BITS, G, MIXED>(a, b0, nblk, col0, smem, bars, abort, lane);
+  else grad_consume<XT, BITS, G, NB, CW, MIXED>(a, warp, b0, nblk, smem, bars, abort, lane, acc);
   __syncthreads();  // ring drained: reuse it for the cross-warp sums
 
   // red[warp row group][token][column]: warps w and w + 1 (CW = 2) cover the

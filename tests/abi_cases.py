@@ -105,7 +105,8 @@ def test_linear_grad_input_validation(L):
     assert grad(L, M=-1) == bq.BQ_ERR_SHAPE
     assert grad(L, dt=bq.BQ_F32) == bq.BQ_ERR_UNSUPPORTED
     assert grad(L, layout=0) == bq.BQ_ERR_UNSUPPORTED       # reads the interleaved layout
-    assert grad(L, bm=FAKE) == bq.BQ_ERR_UNSUPPORTED        # uniform width only
+    assert grad(L, bm=FAKE, N=4000) == bq.BQ_ERR_SHAPE      # a width map needs whole 128-row blocks
+    assert grad(L, bm=FAKE, K=4160) == bq.BQ_ERR_SHAPE      # 128-column slices
     assert grad(L, bits=3) == bq.BQ_ERR_UNSUPPORTED
     assert grad(L, group=16) == bq.BQ_ERR_UNSUPPORTED
     assert grad(L, N=24) == bq.BQ_ERR_SHAPE                 # row tiles of 16
