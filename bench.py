@@ -441,6 +441,31 @@ def mixed_numbers(layers, Ms, hbm, reps=5):
             per_m[str(M)] = {"ms": round(t * 1e3, 4), "GBps": round(byts / t / 1e9, 1),
                              "frac_of_measured_hbm": round(byts / t / 1e9 / hbm, 4)}
             del g
+            # the input gradient dx = dy . dequant(W) of the same linears
+            dys = {N: synth.activations(M, N, seed=8, device="cuda") for N in {m[0] for m in mods}}
+            dxs = {K: torch.empty((M, K), dtype=torch.bfloat16, device="cuda") for K in {m[1] for m in mods}}
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(s):
+                for (N, K, pk, sc, ze, bm, *_rest) in mods[:4]:   # lazy init outside the capture
+                    bq.bq_linear_grad_input(dys[N], pk, sc, ze, K, out=dxs[K], stream=s, bit_map_dev=bm)
+                s.synchronize()
+                with torch.cuda.graph(g, stream=s):
+                    for (N, K, pk, sc, ze, bm, *_rest) in mods:
+                        bq.bq_linear_grad_input(dys[N], pk, sc, ze, K, out=dxs[K], stream=s, bit_map_dev=bm)
+            g.replay()
+            torch.cuda.synchronize()
+            ts = []
+            for _ in range(reps):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                g.replay()
+                b.record()
+                b.synchronize()
+                ts.append(a.elapsed_time(b) / 1e3)
+            t = statistics.median(ts)
+            per_m[str(M)]["grad_input"] = {"ms": round(t * 1e3, 4), "GBps": round(byts / t / 1e9, 1),
+                                           "frac_of_measured_hbm": round(byts / t / 1e9 / hbm, 4)}
+            del g
         if bq.bq_device_status() != bq.BQ_OK:
             raise RuntimeError("mixed linear reported a device error")
         res[kind] = {"bpw_codes": round((4 * weights4 + 2 * (weights - weights4)) / weights, 4), "launches": len(mods),
