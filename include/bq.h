@@ -243,6 +243,38 @@ bq_status bq_linear(const void *x, bq_dtype xtype, int64_t M, int64_t K,
                     bq_layout layout, void *y, void *stream);
 
 /*
+ * bq_linear_workspace_bytes: device workspace that lets bq_linear_ws split
+ * the K dimension of the tensor-core kernel (M >= 64) for this shape; 0
+ * when no split is planned (bq_linear_ws then does what bq_linear does).
+ * A split is planned when the output tiles (128 weight rows x 256 tokens)
+ * would occupy fewer than half of the SMs: SK CTAs (2..8, filling one wave)
+ * then share each tile, each over a K range of whole code stages (256
+ * columns at 4 bits, 512 at 2 bits or under a width map).  The workspace
+ * holds their fp32 partial tiles (128 KB per CTA) and one counter per tile.
+ *   mixed    nonzero for a width map (bits then ignored)
+ * Returns 0 for shapes the tensor-core kernel does not take.
+ */
+size_t bq_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits, int mixed);
+
+/*
+ * bq_linear_ws: bq_linear with a DEVICE workspace for the split-K plan of
+ * bq_linear_workspace_bytes.  A NULL or smaller workspace disables the split
+ * (the result is then bq_linear's).  With a split, each CTA stores its
+ * partial tile and counts its arrival; the CTA that arrives last adds the
+ * partials in rank order and writes y, so y is deterministic (it can differ
+ * from bq_linear's in the last bits: another fp32 summation order).  The
+ * library resets the counters it uses at each call (on `stream`, before the
+ * kernel); two calls in flight at the same time must not share a workspace.
+ *   workspace  256-byte aligned (BQ_ERR_ALIGN otherwise)
+ * Other arguments, rules and errors as bq_linear.  No page describes a
+ * split of the contraction: it is a scheduling choice of this library.
+ */
+bq_status bq_linear_ws(const void *x, bq_dtype xtype, int64_t M, int64_t K,
+                       const void *packed, const float *scales, const uint8_t *zeros,
+                       const uint8_t *bit_map, int bits, int group, int64_t N,
+                       bq_layout layout, void *y, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * bq_linear_f16s: bq_linear for weights from bq_quantize_f16s (binary16
  * scales, uniform width, bits 4 with group 128 or bits 2 with group 64; no
  * bit map).  The binary16 scale is exact in fp32, so the products are

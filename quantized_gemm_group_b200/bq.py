@@ -34,7 +34,7 @@ EXPORTS = (
     "bq_packed_bytes", "bq_group_count", "bq_mixed_offsets", "bq_quantize", "bq_quantize_symmetric",
     "bq_quantize_mixed",
     "bq_dequantize", "bq_fake_quantize", "bq_linear", "bq_linear_grad_input", "bq_check_division",
-    "bq_check_const_division", "bq_quantize_f16s", "bq_linear_f16s",
+    "bq_check_const_division", "bq_quantize_f16s", "bq_linear_f16s", "bq_linear_workspace_bytes", "bq_linear_ws",
     "bq_selftest_bounded_wait", "bq_set_option", "bq_get_option", "bq_device_status",
     "bq_status_string", "bq_version",
 )
@@ -83,6 +83,10 @@ def lib(path: str | None = None):
     L.bq_linear.restype = i32
     L.bq_linear_f16s.argtypes = [vp, i32, i64, i64, vp, vp, vp, i32, i32, i64, i32, vp, vp]
     L.bq_linear_f16s.restype = i32
+    L.bq_linear_workspace_bytes.argtypes = [i64, i64, i64, i32, i32]
+    L.bq_linear_workspace_bytes.restype = ctypes.c_size_t
+    L.bq_linear_ws.argtypes = [vp, i32, i64, i64, vp, vp, vp, vp, i32, i32, i64, i32, vp, vp, ctypes.c_size_t, vp]
+    L.bq_linear_ws.restype = i32
     L.bq_linear_grad_input.argtypes = [vp, i32, i64, i64, vp, vp, vp, vp, i32, i32, i64, i32, vp, vp]
     L.bq_linear_grad_input.restype = i32
     L.bq_check_division.argtypes = [ctypes.c_uint32, ctypes.c_uint32, i32, vp, vp]
@@ -216,10 +220,16 @@ def bq_fake_quantize(W: torch.Tensor, bits: int, group: int | None = None, out_d
     return o
 
 
+def bq_linear_workspace_bytes(M: int, N: int, K: int, bits: int = 4, mixed: bool = False) -> int:
+    """Device workspace bytes that let bq_linear(..., workspace=...) split K (0: no split)."""
+    return int(lib().bq_linear_workspace_bytes(M, N, K, bits, 1 if mixed else 0))
+
+
 def bq_linear(x: torch.Tensor, packed, scales, zeros, N: int, bits: int = 4, group: int | None = None,
-              bit_map_dev=None, layout: str = "interleaved", out=None, stream=None):
+              bit_map_dev=None, layout: str = "interleaved", out=None, stream=None, workspace=None):
     """y [M, N] = x [M, K] . dequant(W)^T, y in x's dtype.  fp16 `scales` (from the binary16
-    scale format) select bq_linear_f16s."""
+    scale format) select bq_linear_f16s; a device `workspace` (uint8, from
+    bq_linear_workspace_bytes) selects bq_linear_ws."""
     group = group or GROUP_OF_BITS.get(bits, 0)
     M, K = x.shape
     y = out if out is not None else torch.empty((M, N), dtype=x.dtype, device=x.device)
@@ -229,6 +239,12 @@ def bq_linear(x: torch.Tensor, packed, scales, zeros, N: int, bits: int = 4, gro
         st = lib().bq_linear_f16s(_ptr(x), DTYPE_CODE[x.dtype], M, K, _ptr(packed), _ptr(scales), _ptr(zeros),
                                   bits, group, N, LAYOUTS[layout], _ptr(y), _stream(stream))
         _check("bq_linear_f16s", st)
+        return y
+    if workspace is not None:
+        st = lib().bq_linear_ws(_ptr(x), DTYPE_CODE[x.dtype], M, K, _ptr(packed), _ptr(scales), _ptr(zeros),
+                                _ptr(bit_map_dev), bits, group, N, LAYOUTS[layout], _ptr(y), _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), _stream(stream))
+        _check("bq_linear_ws", st)
         return y
     st = lib().bq_linear(_ptr(x), DTYPE_CODE[x.dtype], M, K, _ptr(packed), _ptr(scales), _ptr(zeros),
                          _ptr(bit_map_dev), bits, group, N, LAYOUTS[layout], _ptr(y), _stream(stream))

@@ -502,7 +502,7 @@ bool make_x_map(CUtensorMap *map, const uint16_t *x, int64_t M, int64_t K, int x
 }
 
 template <int XT, int BITS, int G, bool MIXED = false, bool S16 = false>
-bq_status launch_gemm_t(const uint16_t *x, int64_t M, int64_t K, const GemmArgs &a, cudaStream_t st) {
+bq_status launch_gemm_t(const uint16_t *x, int64_t M, int64_t K, const GemmArgs &a, int SK, cudaStream_t st) {
   auto kern = gemm_kernel<XT, BITS, G, MIXED, S16>;
   // the warpgroups' setmaxnreg shares must fit in the registers the block is
   // launched with, or the raising warpgroups would wait forever (a property
@@ -518,7 +518,10 @@ bq_status launch_gemm_t(const uint16_t *x, int64_t M, int64_t K, const GemmArgs 
   CUtensorMap map;
   if (!make_x_map(&map, x, M, K, XT)) return BQ_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(a.N / kGemmRowTile), (unsigned)((M + kGemmTokTile - 1) / kGemmTokTile), 1);
+  const unsigned tiles_x = (unsigned)(a.N / kGemmRowTile), tiles_y = (unsigned)((M + kGemmTokTile - 1) / kGemmTokTile);
+  if (SK > 1 && cudaMemsetAsync(a.ws_ctr, 0, (size_t)tiles_x * tiles_y * sizeof(unsigned), st) != cudaSuccess)
+    return BQ_ERR_CUDA;
+  cfg.gridDim = dim3(tiles_x, tiles_y, (unsigned)SK);
   cfg.blockDim = dim3(kGemmThreads, 1, 1);
   cfg.dynamicSmemBytes = (size_t)GemmSmem::total;
   cfg.stream = st;
@@ -546,10 +549,36 @@ bool gemm_eligible(int64_t M, int64_t N, const uint8_t *bit_map, int group) {
          M <= 65535LL * kGemmTokTile;
 }
 
+// Split-K plan of the tensor-core kernel: when the output tiles (128 rows x
+// 256 tokens) fill fewer than half of the SMs, SK CTAs share each tile, each
+// a K range of whole code stages (256 columns at 4 bits, 512 at 2 bits or
+// under a width map), so that tiles x SK fills one wave (SK <= 8).  The
+// partial tiles and per-tile counters live in the caller's workspace.
+struct GemmSplit {
+  int SK, unit;
+  int64_t tiles;
+  size_t part_bytes, bytes;
+};
+
+GemmSplit gemm_split_plan(int64_t M, int64_t N, int64_t K, int bits, bool mixed) {
+  GemmSplit p;
+  p.unit = (mixed || bits == 2) ? 512 : 256;
+  p.tiles = (N / kGemmRowTile) * ((M + kGemmTokTile - 1) / kGemmTokTile);
+  const int64_t sms = sm_count();
+  int64_t sk = (p.tiles > 0) ? sms / p.tiles : 1;
+  if (sk > 8) sk = 8;
+  if (sk > K / p.unit) sk = K / p.unit;
+  if (2 * p.tiles > sms || sk < 2 || K % p.unit) sk = 1;
+  p.SK = (int)sk;
+  p.part_bytes = (size_t)p.tiles * sk * kGemmTokTile * kGemmRowTile * sizeof(float);
+  p.bytes = (p.SK > 1) ? p.part_bytes + (size_t)p.tiles * sizeof(unsigned) : 0;
+  return p;
+}
+
 template <int XT>
 bq_status gemm_dispatch(const uint16_t *x, int64_t M, int64_t K, const uint8_t *packed, const void *scales, bool s16,
                         const uint8_t *zeros, const uint8_t *bit_map, int bits, int group, int64_t N, uint16_t *y,
-                        cudaStream_t st) {
+                        void *workspace, size_t workspace_bytes, cudaStream_t st) {
   GemmArgs a = {};
   a.packed = packed;
   a.scales = scales;
@@ -559,15 +588,23 @@ bq_status gemm_dispatch(const uint16_t *x, int64_t M, int64_t K, const uint8_t *
   a.M = M;
   a.K = K;
   a.N = N;
+  const GemmSplit sp = gemm_split_plan(M, N, K, bits, bit_map != nullptr);
+  int SK = 1;
+  if (sp.SK > 1 && workspace && workspace_bytes >= sp.bytes) {
+    SK = sp.SK;
+    a.ws_part = reinterpret_cast<float *>(workspace);
+    a.ws_ctr = reinterpret_cast<unsigned *>(reinterpret_cast<char *>(workspace) + sp.part_bytes);
+    a.split_unit = sp.unit;
+  }
   if (s16) {
     if (bit_map) return BQ_ERR_UNSUPPORTED;
-    if (bits == 4 && group == 128) return launch_gemm_t<XT, 4, 128, false, true>(x, M, K, a, st);
-    if (bits == 2 && group == 64) return launch_gemm_t<XT, 2, 64, false, true>(x, M, K, a, st);
+    if (bits == 4 && group == 128) return launch_gemm_t<XT, 4, 128, false, true>(x, M, K, a, SK, st);
+    if (bits == 2 && group == 64) return launch_gemm_t<XT, 2, 64, false, true>(x, M, K, a, SK, st);
     return BQ_ERR_UNSUPPORTED;
   }
-  if (bit_map) return launch_gemm_t<XT, 4, 128, true>(x, M, K, a, st);
+  if (bit_map) return launch_gemm_t<XT, 4, 128, true>(x, M, K, a, SK, st);
 #define BQ_GM(B, G_) \
-  if (bits == B && group == G_) return launch_gemm_t<XT, B, G_>(x, M, K, a, st);
+  if (bits == B && group == G_) return launch_gemm_t<XT, B, G_>(x, M, K, a, SK, st);
   BQ_GM(4, 128) BQ_GM(2, 64) BQ_GM(4, 64) BQ_GM(4, 256) BQ_GM(2, 128) BQ_GM(2, 256)
 #undef BQ_GM
   return BQ_ERR_UNSUPPORTED;
@@ -767,10 +804,11 @@ bq_status bq_fake_quantize(const void *W, bq_dtype wtype, int64_t rows, int64_t 
 
 namespace {
 
-// bq_linear and bq_linear_f16s: s16 selects binary16 scales.
+// bq_linear, bq_linear_f16s and bq_linear_ws: s16 selects binary16 scales;
+// a workspace lets the tensor-core kernel split K (see gemm_split_plan).
 bq_status linear_any(const void *x, bq_dtype xtype, int64_t M, int64_t K, const void *packed, const void *scales,
                      bool s16, const uint8_t *zeros, const uint8_t *bit_map, int bits, int group, int64_t N,
-                     bq_layout layout, void *y, void *stream) {
+                     bq_layout layout, void *y, void *stream, void *workspace = nullptr, size_t workspace_bytes = 0) {
   if (M < 0 || K < 0 || N < 0) return BQ_ERR_SHAPE;
   if (s16 && (bit_map || !((bits == 4 && group == 128) || (bits == 2 && group == 64)))) return BQ_ERR_UNSUPPORTED;
   if (xtype != BQ_F16 && xtype != BQ_BF16) return BQ_ERR_UNSUPPORTED;
@@ -795,8 +833,11 @@ bq_status linear_any(const void *x, bq_dtype xtype, int64_t M, int64_t K, const 
   uint16_t *yy = reinterpret_cast<uint16_t *>(y);
   const uint8_t *pk = reinterpret_cast<const uint8_t *>(packed);
   if (gemm_eligible(M, N, bit_map, group))
-    return (xtype == BQ_BF16) ? gemm_dispatch<1>(xx, M, K, pk, scales, s16, zeros, bit_map, bits, group, N, yy, st)
-                              : gemm_dispatch<0>(xx, M, K, pk, scales, s16, zeros, bit_map, bits, group, N, yy, st);
+    return (xtype == BQ_BF16)
+               ? gemm_dispatch<1>(xx, M, K, pk, scales, s16, zeros, bit_map, bits, group, N, yy, workspace,
+                                  workspace_bytes, st)
+               : gemm_dispatch<0>(xx, M, K, pk, scales, s16, zeros, bit_map, bits, group, N, yy, workspace,
+                                  workspace_bytes, st);
   // Otherwise token blocks of at most 16 go through the decode kernel.
   for (int64_t m0 = 0; m0 < M; m0 += 16) {
     const int mb = (int)((M - m0) < 16 ? (M - m0) : 16);
@@ -824,6 +865,19 @@ bq_status bq_linear_f16s(const void *x, bq_dtype xtype, int64_t M, int64_t K, co
                          const uint16_t *scales, const uint8_t *zeros, int bits, int group, int64_t N,
                          bq_layout layout, void *y, void *stream) {
   return linear_any(x, xtype, M, K, packed, scales, true, zeros, nullptr, bits, group, N, layout, y, stream);
+}
+
+size_t bq_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits, int mixed) {
+  if (M < kGemmMinTokens || N <= 0 || K <= 0 || N % kGemmRowTile) return 0;
+  return gemm_split_plan(M, N, K, bits, mixed != 0).bytes;
+}
+
+bq_status bq_linear_ws(const void *x, bq_dtype xtype, int64_t M, int64_t K, const void *packed, const float *scales,
+                       const uint8_t *zeros, const uint8_t *bit_map, int bits, int group, int64_t N,
+                       bq_layout layout, void *y, void *workspace, size_t workspace_bytes, void *stream) {
+  if (workspace && !aligned(workspace, 256)) return BQ_ERR_ALIGN;
+  return linear_any(x, xtype, M, K, packed, scales, false, zeros, bit_map, bits, group, N, layout, y, stream,
+                    workspace, workspace_bytes);
 }
 
 bq_status bq_linear_grad_input(const void *dy, bq_dtype dtype, int64_t M, int64_t N, const void *packed,

@@ -94,6 +94,7 @@ struct GemmSmem {
   static constexpr int epi_off = xprog_off + 4;                      // releases of TMEM buffer 0, 1
   static constexpr int tmem_off = epi_off + 8 + 4;
   static constexpr int abort_off = tmem_off + 8;
+  static constexpr int last_off = abort_off + 4;       // split-K: this CTA arrived last
   static constexpr int total = abort_off + 8 + 1024;   // + alignment slack
 };
 
@@ -104,6 +105,15 @@ struct GemmArgs {
   const uint8_t *bit_map;
   uint16_t *y;
   int64_t M, K, N;
+  // split-K (gridDim.z CTAs per output tile, each a K range of whole
+  // `split_unit`-column units): fp32 partial tiles [tile][rank][token][row]
+  // and one arrival counter per tile (zero before the launch); unused when
+  // gridDim.z == 1.  Inside the roles K is the CTA's range and k0x its first
+  // column in x.
+  float *ws_part;
+  unsigned *ws_ctr;
+  int split_unit;
+  int64_t k0x;
 };
 
 // Shared-memory addresses of the mbarriers.
@@ -245,7 +255,8 @@ BQ_DEV void gemm_produce(const GemmArgs &a, const CUtensorMap *xmap, const uint8
       if (ci < kGemmXStages || mbar_test_wait(B.empty + 8u * st, ((ci / kGemmXStages) & 1) ^ 1)) {
         const uint32_t full = B.full + 8u * st;
         mbar_arrive_expect_tx(full, (uint32_t)GemmSmem::X_BYTES);
-        tma_load_2d(sbase + GemmSmem::x_off + st * GemmSmem::X_BYTES, xmap, ci * kGemmChunk, tok0, full);
+        tma_load_2d(sbase + GemmSmem::x_off + st * GemmSmem::X_BYTES, xmap, (int)(a.k0x + ci * kGemmChunk), tok0,
+                    full);
         ++ci;
         progress = true;
       }
@@ -460,15 +471,63 @@ BQ_DEV void gemm_epilogue(const GemmArgs &a, const void *sc, int e, int warp, in
     __syncwarp();
     if (lane == 0) red_release_add(epi + 4u * buf, 1u);  // buffer g & 1 is free again
   }
-  if (!ok || *abort) return;
+  const int SK = (int)gridDim.z;
   // y is [M][N], token-major; this thread owns row (row0 + rloc)
   const int64_t n = row0 + rloc;
-#pragma unroll 8
+  if (SK == 1) {
+    if (!ok || *abort) return;
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+      const int64_t tok = tok0 + col0 + i;
+      if (tok < a.M)
+        a.y[tok * a.N + n] = XT ? __bfloat16_as_ushort(__float2bfloat16_rn(acc[i])) : __half_as_ushort(__float2half_rn(acc[i]));
+    }
+    return;
+  }
+  // Split-K: store this CTA's partial tile (token-major, so a warp's 32 rows
+  // of one token are one 128-byte line), fence, and count the arrival; the
+  // CTA that arrives last sums the partials in rank order and writes y.  No
+  // CTA waits for another.  Every epilogue warp reaches both barriers, also
+  // after a timeout (which then skips the arrival, so no CTA writes y).
+  const int64_t tile = blockIdx.x + (int64_t)blockIdx.y * gridDim.x;
+  const int rank = (int)blockIdx.z;
+  const bool good = ok && !*abort;
+  (void)rank;
+  float *mine = a.ws_part + (tile * SK + rank) * (int64_t)(kGemmTokTile * kGemmRowTile);
+  if (good) {
+#pragma unroll
+    for (int i = 0; i < 64; ++i) mine[(col0 + i) * kGemmRowTile + rloc] = acc[i];
+  }
+  __threadfence();
+  asm volatile("bar.sync 1, %0;" ::"n"(kGemmEpiWarps * 32) : "memory");
+  const uint32_t lastw = sbase + GemmSmem::last_off;
+  if (e == 0 && lane == 0) {
+    uint32_t is_last = 0;
+    if (!*abort) is_last = (atomicAdd(a.ws_ctr + tile, 1u) == (unsigned)(SK - 1)) ? 1u : 0u;
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(lastw), "r"(is_last) : "memory");
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(kGemmEpiWarps * 32) : "memory");
+  uint32_t is_last;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(is_last) : "r"(lastw) : "memory");
+  if (!is_last) return;
+  __threadfence();
+  // every rank's partial (this CTA's own included) from the workspace, in
+  // rank order; the 64 loads of one rank are independent of each other
+  const float *parts = a.ws_part + tile * SK * (int64_t)(kGemmTokTile * kGemmRowTile) + col0 * kGemmRowTile + rloc;
+#pragma unroll
+  for (int i = 0; i < 64; ++i) acc[i] = __ldcg(parts + i * kGemmRowTile);
+  for (int q = 1; q < SK; ++q) {
+    const float *pq = parts + (int64_t)q * (kGemmTokTile * kGemmRowTile);
+#pragma unroll
+    for (int i = 0; i < 64; ++i) acc[i] += __ldcg(pq + i * kGemmRowTile);
+  }
+#pragma unroll
   for (int i = 0; i < 64; ++i) {
     const int64_t tok = tok0 + col0 + i;
     if (tok < a.M)
       a.y[tok * a.N + n] = XT ? __bfloat16_as_ushort(__float2bfloat16_rn(acc[i])) : __half_as_ushort(__float2half_rn(acc[i]));
   }
+  if (e == 0 && lane == 0) a.ws_ctr[tile] = 0u;  // ready for the next call
 }
 
 // The roles of one CTA for a block of width BITS, group G.
@@ -574,9 +633,23 @@ gemm_kernel(const __grid_constant__ CUtensorMap xmap, const GemmArgs a) {
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // split-K: this CTA's K range, whole units of split_unit columns, and its
+  // block's codes / scales / zeros from the range's first column
+  GemmArgs al = a;
+  if (gridDim.z > 1) {
+    const int64_t SK = gridDim.z, nu = a.K / a.split_unit;
+    const int64_t k0 = (blockIdx.z * nu / SK) * a.split_unit, k1 = ((blockIdx.z + 1) * nu / SK) * a.split_unit;
+    const int bb = MIXED ? bits : BITS;
+    const int gsz = (!MIXED || bits == BITS) ? G : 64;
+    pk += k0 * 16 * bb;  // 128 rows x k0 columns x bb / 8 bytes
+    sc += (k0 / gsz) * kGemmRowTile * SB;
+    ze += (k0 / gsz) * kGemmRowTile;
+    al.K = k1 - k0;
+    al.k0x = k0;
+  }
   pdl_wait();
-  if (!MIXED || bits == BITS) gemm_roles<XT, BITS, G, S16>(a, &xmap, pk, sc, ze, warp, lane, tmem, sbase, B, abort, row0, tok0);
-  else gemm_roles<XT, 2, 64, S16>(a, &xmap, pk, sc, ze, warp, lane, tmem, sbase, B, abort, row0, tok0);
+  if (!MIXED || bits == BITS) gemm_roles<XT, BITS, G, S16>(al, &xmap, pk, sc, ze, warp, lane, tmem, sbase, B, abort, row0, tok0);
+  else gemm_roles<XT, 2, 64, S16>(al, &xmap, pk, sc, ze, warp, lane, tmem, sbase, B, abort, row0, tok0);
 
   // everything issued by this CTA has finished before the tensor memory goes
   tc_fence_before();
