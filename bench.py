@@ -618,6 +618,55 @@ GEMM_SHAPES = ((14336, 4096), (4096, 14336), (49152, 8192), (8192, 49152))
 GEMM_M = (2048, 4096, 8192)
 
 
+def medium_m_numbers(reps=20):
+    """Medium token counts (the prefill of short prompts, batched decode):
+    bq_linear at M = 32 (two 16-token decode passes) and M = 64 .. 256 (the
+    tensor-core kernel, split over K through bq_linear_ws's workspace where
+    the plan splits), INT4 g128 on Llama-3-8B shapes, one CUDA graph of 8
+    calls per point, CUDA-event median; TFLOP/s = 2 M N K / time."""
+    res = {}
+    s = torch.cuda.Stream()
+    for (N, K) in ((4096, 4096), (6144, 4096), (28672, 4096), (4096, 14336)):
+        W = synth.normal((N, K), 0.02, seed=N + 3 * K, dtype="f16", device="cuda")
+        pk, sc, ze = bq.bq_quantize(W, 4, 128, "interleaved")
+        del W
+        for M in (32, 64, 128, 256):
+            x = synth.activations(M, K, seed=M + 1, device="cuda")
+            y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+            wsb = bq.bq_linear_workspace_bytes(M, N, K, 4)
+            ws = torch.empty(wsb, dtype=torch.uint8, device="cuda") if wsb else None
+            with torch.cuda.stream(s):
+                bq.bq_linear(x, pk, sc, ze, N, 4, 128, out=y, stream=s, workspace=ws)
+                s.synchronize()
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=s):
+                    for _ in range(8):
+                        bq.bq_linear(x, pk, sc, ze, N, 4, 128, out=y, stream=s, workspace=ws)
+            with torch.cuda.stream(s):
+                g.replay()
+            s.synchronize()
+            ts = []
+            for _ in range(reps):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                with torch.cuda.stream(s):
+                    a.record(s)
+                    g.replay()
+                    b.record(s)
+                b.synchronize()
+                ts.append(a.elapsed_time(b) / 1e3 / 8)
+            t = statistics.median(ts)
+            path = "decode passes" if M < 64 else (f"tensor cores, split-K ({wsb // 1024} KB workspace)" if wsb
+                                                   else "tensor cores")
+            res[f"{N}x{K} M{M}"] = {"us": round(t * 1e6, 1), "TFLOPs": round(2.0 * M * N * K / t / 1e12, 1),
+                                    "path": path}
+            del g, x, y, ws
+        del pk, sc, ze
+        torch.cuda.empty_cache()
+    if bq.bq_device_status() != bq.BQ_OK:
+        raise RuntimeError("linear reported a device error")
+    return res
+
+
 def gemm_numbers(Ms, bf16, bf16_sus, reps=10):
     """Prefill weight-only GEMM (tcgen05 path of bq_linear) at the prefill
     shapes: bf16 x N(0,1) [M, K] against INT4 g128 / INT2 g64 weights
@@ -849,6 +898,7 @@ def run_gpu(args, world, rank, local):
         extra["quantizer_8192x49152"] = quant_shape_numbers(hbm)
     if not args.no_gemm:
         extra["prefill_gemm"] = gemm_numbers(GEMM_M if not args.quick else (2048,), bf16, bf16_sus or bf16)
+        extra["medium_m"] = medium_m_numbers()
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(t_step * 1e3, 4), "higher_is_better": True,
